@@ -1,0 +1,200 @@
+/*
+ * sq.h — C ABI of libsq: a W8A8 INT8 quantized linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer computes Y = dequant( int8(X * diag(s)^-1) . int8(diag(s) * W)^T ) + bias
+ * (SmoothQuant smoothing, symmetric absmax INT8 quantization, INT8 x INT8 -> INT32
+ * accumulation, per-token x per-channel/per-tensor dequantization), and the
+ * LLM.int8() decomposition in which activation columns whose absmax exceeds a
+ * threshold go through a bf16 product that is added back.
+ *
+ * Pages the operations follow (cited by title and section):
+ *   [BASICS]  "量化基础与INT8" (quantization fundamentals and INT8)
+ *   [LLMINT8] "LLM.int8()技术解析：8位量化如何优化大语言模型计算"
+ *   [SQ]      "SmoothQuant量化实战：W8A8推理部署与单节点530B模型落地"
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE memory owned by the caller; the library keeps no
+ *     reference to them after the call returns and allocates no memory itself. Where
+ *     an operation needs scratch space the caller passes it (ws, ws_bytes), sized by
+ *     sq_workspace_size().
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream). Results
+ *     are ready once the stream is synchronised.
+ *   - Matrices are row-major. bf16 values are passed as their 16-bit patterns
+ *     (`const void*`). X is [M, K] (tokens x in-features) with leading dimension ldx
+ *     (elements); W is [N, K] (out-features x in-features, the nn.Linear layout) with
+ *     leading dimension ldw. Int8 code matrices Xq [M, K] and Wq [N, K] and the output
+ *     Y [M, N] are dense (leading dimension K, K and N).
+ *   - Shape limits: 1 <= M, N <= 2^31-1; 16 <= K <= 65536 with K % 16 == 0 (so that
+ *     |acc| <= K*128*128 < 2^31 and every row is a whole number of 16-byte vectors);
+ *     ldx, ldw >= K and multiples of 8; N % 8 == 0 for outputs.
+ *   - Alignment: every tensor base 16-byte aligned (float vectors included).
+ *   - Arguments are validated before anything is launched; a violation returns
+ *     SQ_ERR_INVALID / SQ_ERR_ALIGN / SQ_ERR_WORKSPACE, launches nothing and leaves
+ *     outputs untouched. sq_last_error() then gives a message (thread-local).
+ *   - NaN or Inf inputs are outside the contract (outputs undefined, no error).
+ *   - Rounding: codes use round-half-to-even of (value * (127/absmax)) in fp32 and are
+ *     clamped to [-128, 127]; absmax == 0 gives codes 0 and scale 0. The reciprocal
+ *     127/absmax and the scale absmax/127 are IEEE fp32 divisions.
+ */
+#ifndef SQ_H
+#define SQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SQ_API __attribute__((visibility("default")))
+#else
+#define SQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sq_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+  SQ_OK = 0,
+  SQ_ERR_INVALID = -1,     /* null pointer, bad size, bad enum */
+  SQ_ERR_ALIGN = -2,       /* pointer or leading dimension not aligned as required */
+  SQ_ERR_CUDA = -3,        /* a CUDA runtime / driver call failed (message has the code) */
+  SQ_ERR_TIMEOUT = -4,     /* a bounded device-side wait gave up (see sq_sync_status) */
+  SQ_ERR_WORKSPACE = -5,   /* ws NULL or smaller than sq_workspace_size() */
+  SQ_ERR_UNSUPPORTED = -6  /* no sm_100a device, or the library was built without it */
+} sq_status;
+
+typedef enum { SQ_PER_TENSOR = 0, SQ_PER_CHANNEL = 1 } sq_gran;
+
+typedef enum {
+  SQ_OP_SMOOTH_QUANT_WEIGHT = 1,
+  SQ_OP_INT8_GEMM_DEQUANT = 2,
+  SQ_OP_LLMINT8 = 3
+} sq_op;
+
+/*
+ * Per-input-channel absolute maximum of the activations (calibration statistic).
+ *   amax[j] = max_m |X[m, j]|                  (accumulate == 0)
+ *   amax[j] = max(amax[j], max_m |X[m, j]|)    (accumulate != 0: running maximum
+ *                                               over calibration batches)
+ * [SQ] §3.2 (forward hook: x.abs().amax over the token dimensions, torch.maximum
+ * across batches); [LLMINT8] §2.1 step 1 (column-wise absolute maximum).
+ * X: bf16 [M, K], ldx. amax: fp32 [K], read (accumulate) and written. Exact (a max).
+ */
+SQ_API sq_status sq_act_channel_absmax(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, float* amax,
+                                int accumulate, sq_stream_t stream);
+
+/*
+ * SmoothQuant smoothing factors. [SQ] §2.1 (s_j = max|X_j|^alpha / max|W_j|^(1-alpha))
+ * and §3.3 (weight maximum over the output dimension, both maxima clamped at 1e-8):
+ *   wmax_j  = max_n |W[n, j]|
+ *   s_j     = fp32( pow(max(act_amax_j,1e-8), alpha) / pow(max(wmax_j,1e-8), 1-alpha) )
+ *             (evaluated in fp64, rounded once)
+ *   inv_s_j = 1 / s_j   (fp32)
+ * act_amax: fp32 [K] (from sq_act_channel_absmax). W: bf16 [N, K], ldw.
+ * alpha in [0, 1]. s, inv_s: fp32 [K], written (s may not alias act_amax).
+ */
+SQ_API sq_status sq_smooth_scale(const float* act_amax, const void* W_bf16, int64_t N, int64_t K, int64_t ldw,
+                          float alpha, float* s, float* inv_s, sq_stream_t stream);
+
+/*
+ * Smoothed weight quantization. [SQ] §3.3 (W' = W * s over the input dimension) and
+ * §3.4 (w_scale = max|W'|/127); [BASICS] per-tensor / per-channel granularity and the
+ * quantization-flow example:
+ *   w'[n,k] = W[n,k] * s[k]       (fp32, never rounded; s == NULL means s = 1)
+ *   SQ_PER_CHANNEL: a_n = max_k |w'[n,k]|, w_scale[n] = a_n/127, Wq[n,k] = q(w', a_n)
+ *   SQ_PER_TENSOR : a   = max |w'|,       w_scale[0] = a/127,   Wq[n,k] = q(w', a)
+ *   q(v, a) = clamp(rne(v * (127/a)), -128, 127)
+ * W: bf16 [N, K], ldw. Wq: int8 [N, K] dense. w_scale: fp32 [N] or [1].
+ * ws: SQ_PER_TENSOR needs sq_workspace_size(SQ_OP_SMOOTH_QUANT_WEIGHT, 0, N, K) bytes
+ * (one global maximum); SQ_PER_CHANNEL needs none (ws may be NULL).
+ */
+SQ_API sq_status sq_smooth_quant_weight(const void* W_bf16, int64_t N, int64_t K, int64_t ldw, const float* s,
+                                 sq_gran gran, int8_t* Wq, float* w_scale, void* ws, size_t ws_bytes,
+                                 sq_stream_t stream);
+
+/*
+ * Smoothing + per-token dynamic activation quantization in one pass over X.
+ * [BASICS] per-token granularity and quantization-flow example (X_scale =
+ * X.abs().max(dim=-1)/127); [SQ] §2.3 and §3.4 (divide by s before quantizing,
+ * fused into one light kernel), here as a multiply by inv_s:
+ *   x'[m,k] = X[m,k] * inv_s[k]   (fp32; inv_s == NULL means 1)
+ *   a_m = max_k |x'[m,k]|, x_scale[m] = a_m/127, Xq[m,k] = clamp(rne(x' * (127/a_m)), -128, 127)
+ * X: bf16 [M, K], ldx. Xq: int8 [M, K] dense. x_scale: fp32 [M].
+ */
+SQ_API sq_status sq_quant_act_per_token(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, const float* inv_s,
+                                 int8_t* Xq, float* x_scale, sq_stream_t stream);
+
+/*
+ * INT8 GEMM with fused dequantization epilogue on the 5th-generation tensor cores.
+ * [BASICS] INT8 inference flow ("(M,K) x (K,N) -> INT32 accumulate, INT32 -> 16-bit
+ * dequantized output") and quantization-flow example (Y = Y_int32 * X_scale * W_scale);
+ * [SQ] §3.4 (out * (x_scale * w_scale) + bias, bias kept in floating point, §4.5):
+ *   acc[m,n] = sum_k Xq[m,k] * Wq[n,k]                         (exact int32)
+ *   Y[m,n]   = bf16_rne( (float(acc) * x_scale[m]) * w_scale[n or 0] + bias[n] )
+ * Xq: int8 [M, K]; Wq: int8 [N, K]; x_scale: fp32 [M]; w_scale: fp32 [N] (SQ_PER_CHANNEL)
+ * or [1] (SQ_PER_TENSOR); bias: bf16 [N] or NULL; Y: bf16 [M, N].
+ * acc_out: int32 [M, N] or NULL — when given, the raw INT32 accumulator is written too
+ * (for exact checking). ws: sq_workspace_size(SQ_OP_INT8_GEMM_DEQUANT, M, N, K) bytes
+ * (zero for the shapes that need none; ws may then be NULL).
+ */
+SQ_API sq_status sq_int8_gemm_dequant(const int8_t* Xq, const int8_t* Wq, const float* x_scale, const float* w_scale,
+                               sq_gran w_gran, const void* bias_bf16, void* Y_bf16, int64_t M, int64_t N,
+                               int64_t K, int32_t* acc_out, void* ws, size_t ws_bytes, sq_stream_t stream);
+
+/*
+ * LLM.int8() mixed-precision decomposed linear. [LLMINT8] §2.1 (column absmax of the
+ * input, columns over the threshold are outliers, handled apart; the rest in 8 bits),
+ * §2.2 (quantize / dequantize), §3.1 (bitmask of outlier columns, INT8 GEMM for the
+ * normal columns, 16-bit GEMM for the outlier columns, results merged):
+ *   amax_j = max_m |X[m,j]|;   O = { j : amax_j > threshold }   (strict)
+ *   a_m = max_{k not in O} |X[m,k]|, d_m = a_m/127, Xq[m,k] = q(X[m,k], a_m) for k not in O,
+ *         Xq[m,k] = 0 for k in O
+ *   acc[m,n] = sum_k Xq[m,k] * Wq[n,k]                                  (exact int32)
+ *   o[m,n]   = sum_{j in O} X[m,j] * W[n,j]     (bf16 inputs, fp32 tensor-core accumulate)
+ *   Y[m,n]   = bf16_rne( (float(acc) * d_m) * w_scale[n] + o[m,n] + bias[n] )
+ * X: bf16 [M, K], ldx == K. W: bf16 [N, K], ldw == K (the original weight; its outlier
+ * columns feed the 16-bit product). Wq, w_scale: the per-channel int8 weight and scales
+ * of the UNSMOOTHED W (sq_smooth_quant_weight(W, s = NULL, SQ_PER_CHANNEL)).
+ * bias: bf16 [N] or NULL. Y: bf16 [M, N].
+ * mask_out: uint32 [ceil(K/32)] or NULL (bit j%32 of word j/32 set for j in O).
+ * n_outliers_out: int32 [1] device or NULL (|O|). acc_out: int32 [M, N] or NULL.
+ * ws: sq_workspace_size(SQ_OP_LLMINT8, M, N, K) bytes (holds the int8 activations, the
+ * outlier index list and the gathered outlier columns of X and W).
+ */
+SQ_API sq_status llmint8_decomposed_linear(const void* X_bf16, const void* W_bf16, const int8_t* Wq,
+                                    const float* w_scale, float threshold, const void* bias_bf16, void* Y_bf16,
+                                    int64_t M, int64_t N, int64_t K, uint32_t* mask_out,
+                                    int32_t* n_outliers_out, int32_t* acc_out, void* ws, size_t ws_bytes,
+                                    sq_stream_t stream);
+
+/* Bytes of scratch an operation needs for the given shape (0 if none). Returns 0 for an
+ * unknown op; never fails otherwise. */
+SQ_API size_t sq_workspace_size(int op, int64_t M, int64_t N, int64_t K);
+
+/* Message for the last non-OK status returned on the calling thread ("" if none). The
+ * pointer stays valid until the next call on that thread. */
+SQ_API const char* sq_last_error(void);
+
+/* Synchronises `stream`, then reads and clears the current device's error word, which
+ * kernels set when a bounded wait gives up (a device-side stall or lost arrival) instead
+ * of spinning forever. Returns SQ_OK, SQ_ERR_TIMEOUT or SQ_ERR_CUDA. */
+SQ_API sq_status sq_sync_status(sq_stream_t stream);
+
+/* Library version string and the compute capability it was built for ("sm_100a"). */
+SQ_API const char* sq_version(void);
+
+/* Test hook for the failure path (no counterpart on the pages). Arms the NEXT
+ * sq_int8_gemm_dequant call made on the calling thread: its device-side waits give up after
+ * wait_limit_ns nanoseconds (0 = the default of 2 s) and, when fault == 1, its TMA producer
+ * withholds one pipeline stage, so the consumer's bounded wait runs out. The kernel then
+ * records the timeout, drains its own copies, frees its tensor memory and returns;
+ * sq_sync_status() reports SQ_ERR_TIMEOUT and the context stays usable. Not for production
+ * use; the output of the armed call is undefined. */
+SQ_API void sq_debug_arm_fault(int fault, uint64_t wait_limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_H */

@@ -1,0 +1,105 @@
+"""Helpers for the GPU parity tests: device transfers of bf16 bit patterns, the full
+SmoothQuant and LLM.int8 paths through the C ABI, and the tolerance check."""
+import numpy as np
+import torch
+
+from w8a8_quantized_gemm_b200 import sq
+from w8a8_quantized_gemm_b200 import workloads as wl
+
+DEV = "cuda"
+REL_FROB = 2e-3
+MAX_ABS_REL = 1e-2
+
+
+def dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(DEV)
+
+
+def host_bits(t):
+    return t.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def host(t):
+    return t.detach().cpu().numpy()
+
+
+def empty(shape, dtype):
+    return torch.empty(shape, dtype=dtype, device=DEV)
+
+
+def _sel(t, rows):
+    return t if rows is None else t[torch.as_tensor(rows, device=t.device)]
+
+
+def smoothquant_gpu(p, calib=None, acc=True, s=None, inv_s=None, rows=None, wrows=None):
+    """Run a1..a6 on the GPU through the C ABI. Returns numpy results (only the given
+    activation rows / weight rows of the per-row outputs when `rows` / `wrows` are set)."""
+    X, W = dev_bf16(p.X), dev_bf16(p.W)
+    bias = dev_bf16(p.bias) if p.bias is not None else None
+    M, K, N = p.M, p.K, p.N
+    out = {}
+    if s is None:
+        amax = empty(K, torch.float32)
+        src = dev_bf16(calib) if calib is not None else X
+        sq.sq_act_channel_absmax(src, amax)
+        s_t, inv_t = empty(K, torch.float32), empty(K, torch.float32)
+        sq.sq_smooth_scale(amax, W, p.alpha, s_t, inv_t)
+        out["amax"] = amax
+    else:
+        s_t = torch.from_numpy(s).to(DEV)
+        inv_t = torch.from_numpy(inv_s).to(DEV)
+    Wq = empty((N, K), torch.int8)
+    e = empty(N if p.w_gran == sq.SQ_PER_CHANNEL else 1, torch.float32)
+    ws = sq.workspace(sq.SQ_OP_SMOOTH_QUANT_WEIGHT, 0, N, K)
+    sq.sq_smooth_quant_weight(W, s_t, p.w_gran, Wq, e, ws)
+    Xq = empty((M, K), torch.int8)
+    d = empty(M, torch.float32)
+    sq.sq_quant_act_per_token(X, inv_t, Xq, d)
+    Y = empty((M, N), torch.bfloat16)
+    acc_t = empty((M, N), torch.int32) if acc else None
+    gws = sq.workspace(sq.SQ_OP_INT8_GEMM_DEQUANT, M, N, K)
+    sq.sq_int8_gemm_dequant(Xq, Wq, d, e, p.w_gran, bias, Y, acc_t, gws)
+    sq.sq_sync_status()
+    res = {k: host(v) for k, v in out.items()}
+    e_h = host(e)
+    res.update(s=host(s_t), inv_s=host(inv_t), Wq=host(_sel(Wq, wrows)), e_full=e_h,
+               e=e_h if (wrows is None or e_h.size == 1) else e_h[wrows], Xq=host(_sel(Xq, rows)),
+               d=host(_sel(d, rows)), Y=host_bits(_sel(Y, rows)))
+    if acc:
+        res["acc"] = host(_sel(acc_t, rows))
+    return res
+
+
+def llmint8_gpu(p, threshold=None, acc=True, rows=None):
+    X, W = dev_bf16(p.X), dev_bf16(p.W)
+    bias = dev_bf16(p.bias) if p.bias is not None else None
+    M, K, N = p.M, p.K, p.N
+    Wq = empty((N, K), torch.int8)
+    e = empty(N, torch.float32)
+    sq.sq_smooth_quant_weight(W, None, sq.SQ_PER_CHANNEL, Wq, e)
+    Y = empty((M, N), torch.bfloat16)
+    mask = empty((K + 31) // 32, torch.int32)
+    cnt = empty(1, torch.int32)
+    acc_t = empty((M, N), torch.int32) if acc else None
+    ws = sq.workspace(sq.SQ_OP_LLMINT8, M, N, K)
+    thr = p.threshold if threshold is None else threshold
+    sq.llmint8_decomposed_linear(X, W, Wq, e, thr, bias, Y, mask, cnt, acc_t, ws)
+    sq.sq_sync_status()
+    res = dict(Wq=host(Wq), e=host(e), Y=host_bits(_sel(Y, rows)), mask=host(mask).view(np.uint32),
+               count=int(host(cnt)[0]))
+    if acc:
+        res["acc"] = host(_sel(acc_t, rows))
+    return res
+
+
+def assert_close_bf16(y_bits, y_ref, what=""):
+    """bf16 output vs the fp64 reference: max-abs <= 1e-2 max|ref|, rel-Frobenius <= 2e-3."""
+    y = wl.bf16_bits_to_f32(y_bits).astype(np.float64)
+    ref = np.asarray(y_ref, np.float64)
+    assert np.all(np.isfinite(y)), f"{what}: non-finite output"
+    scale = np.abs(ref).max()
+    err = np.abs(y - ref)
+    frob = np.linalg.norm(y - ref) / max(np.linalg.norm(ref), 1e-300)
+    assert err.max() <= MAX_ABS_REL * scale + 1e-30, f"{what}: max abs err {err.max():.3e} vs {scale:.3e}"
+    assert frob <= REL_FROB, f"{what}: rel Frobenius {frob:.3e}"
+    return float(err.max() / max(scale, 1e-300)), float(frob)

@@ -1,0 +1,80 @@
+// Internal launch interfaces shared by the translation units of libsq.
+// Every launcher returns cudaGetLastError() after enqueueing its work on `stream`.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace sq {
+
+// Bit flags of the per-device error word written by kernels with bounded waits.
+enum : unsigned int {
+  kErrProducerWait = 1u,
+  kErrMmaWait = 2u,
+  kErrEpilogueWait = 4u,
+  kErrTeardownWait = 8u,
+};
+
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s per wait
+
+// Device address of the error word of the current device.
+unsigned int* device_status_word();
+
+// ---- reductions (sq_reduce.cu)
+// Column absmax of a bf16 [rows, K] matrix into amax (fp32 [K], stored as ordered bits).
+// With accumulate == 0 the output is reset first.
+cudaError_t launch_col_absmax(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, float* amax,
+                              bool accumulate, cudaStream_t stream);
+// s/inv_s from act_amax and the column absmax of W already stored in s (in place).
+cudaError_t launch_smooth_factors(const float* act_amax, float* s_inout, float* inv_s, int64_t K, float alpha,
+                                  cudaStream_t stream);
+
+// ---- row quantization (sq_quant.cu)
+struct OutlierView {
+  const uint32_t* mask = nullptr;    // [ceil(K/32)] skip bits (nullptr: no skipping)
+  const int32_t* prefix = nullptr;   // [ceil(K/32)] outliers before each word
+  const int32_t* count = nullptr;    // [1] number of outliers
+  uint16_t* gathered = nullptr;      // [rows, ld_gathered] bf16 outlier values (zero padded to 64)
+  int64_t ld_gathered = 0;
+};
+
+// Per-row smooth + quantize: q[r,k] = clamp(rne(src[r,k]*vec[k] * 127/a_r)), scale[r] = a_r/127.
+cudaError_t launch_quant_rows(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, const float* vec,
+                              const OutlierView& ov, int8_t* q, float* scale, cudaStream_t stream);
+// Per-tensor: global absmax of src*vec into *gmax_bits (reset first), then quantize with it.
+cudaError_t launch_quant_tensor(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, const float* vec,
+                                unsigned int* gmax_bits, int8_t* q, float* scale1, cudaStream_t stream);
+
+// ---- LLM.int8 outlier bookkeeping (sq_outlier.cu)
+cudaError_t launch_outlier_mask(const float* amax, int64_t K, float threshold, uint32_t* mask, int32_t* prefix,
+                                int32_t* idx, int32_t* count, uint32_t* mask_out, int32_t* count_out,
+                                cudaStream_t stream);
+// dst[r, c] = c < count ? src[r, idx[c]] : 0 for c < roundup(count, 64).
+cudaError_t launch_gather_columns(const uint16_t* src, int64_t rows, int64_t ld, const int32_t* idx,
+                                  const int32_t* count, uint16_t* dst, int64_t ld_dst, cudaStream_t stream);
+
+// ---- tensor-core GEMM (sq_gemm.cu)
+struct GemmArgs {
+  const int8_t* Xq = nullptr;       // [M, K]
+  const int8_t* Wq = nullptr;       // [N, K]
+  const float* x_scale = nullptr;   // [M]
+  const float* w_scale = nullptr;   // [N] or [1]
+  bool w_per_channel = true;
+  const uint16_t* bias = nullptr;   // [N] bf16 or nullptr
+  uint16_t* Y = nullptr;            // [M, N] bf16
+  int32_t* acc_out = nullptr;       // [M, N] or nullptr
+  int64_t M = 0, N = 0, K = 0;
+  // LLM.int8 outlier operands (bf16, K-contiguous, leading dimension ld_o), or nullptr.
+  const uint16_t* Xo = nullptr;     // [M, ld_o]
+  const uint16_t* Wo = nullptr;     // [N, ld_o]
+  const int32_t* o_count = nullptr; // [1] number of outlier columns (device)
+  int64_t ld_o = 0;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  uint64_t wait_limit_ns = kDefaultWaitLimitNs;
+  int fault = 0;                    // test hook: 1 = producer withholds one stage
+};
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, bool outliers);
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream, const char** why);
+
+}  // namespace sq

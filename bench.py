@@ -1,0 +1,461 @@
+"""Benchmark of the W8A8 INT8 linear hot path on B200, one JSON line on rank 0.
+
+One step = the whole path on one batch of the Llama-2-7B-shaped MLP up-projection
+(X bf16 [2048, 4096] with 0.1% of the columns scaled x60, W bf16 [11008, 4096]):
+  SmoothQuant linear: channel absmax of X -> smoothing factors (alpha 0.5) -> smoothed
+  per-channel int8 weight -> smoothed per-token int8 activation -> INT8 GEMM + dequant;
+  LLM.int8() linear on the same X and W (threshold 6.0): per-channel int8 of the
+  unsmoothed weight -> decomposed linear (column absmax, outlier mask, masked per-token
+  quantization, gathers, INT8 GEMM with the bf16 outlier product in the same tiles).
+The metric counts the tensor-core work of the two linears (2*M*N*K each, plus
+2*M*N*K_o for the outlier product) per unit of time, whole job over all ranks.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU (torchrun, one rank per GPU): each rank runs its own replica of the workload
+(independent token batches, weak scaling); there is no collective in the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from w8a8_quantized_gemm_b200 import workloads as wl  # noqa: E402
+
+METRIC = "W8A8 linear TOPS and % of B200 INT8 peak; quantize-kernel GB/s vs HBM peak"
+ALPHA = 0.5
+THRESHOLD = 6.0
+N_SETS = 4  # rotating input sets: 4 x (16.8 MB X + 90.2 MB W) = 428 MB > 126 MB L2
+
+# DRAM traffic of one int8 GEMM launch on this workload, from the committed ncu capture
+# (profiles/int8_gemm_llama7b_mlp_up.md), valid while the GEMM source hashes to GEMM_SRC_SHA.
+NCU_GEMM_TRAFFIC_BYTES = None
+GEMM_SRC_SHA = None
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _gemm_src_sha():
+    with open(os.path.join(ROOT, "w8a8_quantized_gemm_b200", "csrc", "sq_gemm.cu"), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Polls NVML (SM clock, clock-event reasons) in a thread during the timed region."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            import torch
+            handle = None
+            try:
+                props = torch.cuda.get_device_properties(device_index)
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.h = handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+
+    def _reasons_now(self):
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return int(fn(self.h))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self._reasons_now()
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml_unavailable"], "samples": 0}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _init_pg(ws, local):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    if ws > 1 and not dist.is_initialized():
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return ws > 1
+
+
+def _max_over_ranks(x: float, use_dist: bool, local: int) -> float:
+    if not use_dist:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=f"cuda:{local}")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(use_dist: bool, local: int):
+    if use_dist:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[local])
+
+
+# ----------------------------------------------------------------------------- our arm
+class Path:
+    """Device buffers and one step of the hot path through the C ABI."""
+
+    def __init__(self, p, dev, n_sets):
+        import torch
+
+        from w8a8_quantized_gemm_b200 import sq
+        self.torch, self.sq, self.p = torch, sq, p
+        M, N, K = p.M, p.N, p.K
+        self.M, self.N, self.K = M, N, K
+
+        def up(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+        self.X = [up(p.X) for _ in range(n_sets)]
+        self.W = [up(p.W) for _ in range(n_sets)]
+        f32, i8 = torch.float32, torch.int8
+        self.amax = torch.empty(K, dtype=f32, device=dev)
+        self.s = torch.empty(K, dtype=f32, device=dev)
+        self.inv_s = torch.empty(K, dtype=f32, device=dev)
+        self.Wq = torch.empty((N, K), dtype=i8, device=dev)
+        self.e = torch.empty(N, dtype=f32, device=dev)
+        self.Xq = torch.empty((M, K), dtype=i8, device=dev)
+        self.d = torch.empty(M, dtype=f32, device=dev)
+        self.Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.Wq0 = torch.empty((N, K), dtype=i8, device=dev)
+        self.e0 = torch.empty(N, dtype=f32, device=dev)
+        self.Y2 = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.cnt = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.ws_gemm = sq.workspace(sq.SQ_OP_INT8_GEMM_DEQUANT, M, N, K, dev)
+        self.ws_llm = sq.workspace(sq.SQ_OP_LLMINT8, M, N, K, dev)
+        self.names = ["act_channel_absmax", "smooth_scale", "smooth_quant_weight", "quant_act_per_token",
+                      "int8_gemm_dequant", "quant_weight_unsmoothed", "llmint8_decomposed_linear"]
+        self.times = {n: 0.0 for n in self.names}
+        self.ev_pool = []
+
+    def step(self, i, record=None):
+        sq, X, W = self.sq, self.X[i % len(self.X)], self.W[i % len(self.W)]
+        ev = []
+
+        def mark():
+            if record is not None:
+                e = self.torch.cuda.Event(enable_timing=True)
+                e.record()
+                ev.append(e)
+
+        mark()
+        sq.sq_act_channel_absmax(X, self.amax)
+        mark()
+        sq.sq_smooth_scale(self.amax, W, ALPHA, self.s, self.inv_s)
+        mark()
+        sq.sq_smooth_quant_weight(W, self.s, sq.SQ_PER_CHANNEL, self.Wq, self.e)
+        mark()
+        sq.sq_quant_act_per_token(X, self.inv_s, self.Xq, self.d)
+        mark()
+        sq.sq_int8_gemm_dequant(self.Xq, self.Wq, self.d, self.e, sq.SQ_PER_CHANNEL, None, self.Y, None, self.ws_gemm)
+        mark()
+        sq.sq_smooth_quant_weight(W, None, sq.SQ_PER_CHANNEL, self.Wq0, self.e0)
+        mark()
+        sq.llmint8_decomposed_linear(X, W, self.Wq0, self.e0, THRESHOLD, None, self.Y2, None, self.cnt, None,
+                                     self.ws_llm)
+        mark()
+        if record is not None:
+            record.append(ev)
+
+    def collect(self, records):
+        self.torch.cuda.synchronize()
+        for ev in records:
+            for j, n in enumerate(self.names):
+                self.times[n] += ev[j].elapsed_time(ev[j + 1])
+        return {n: t / max(len(records), 1) for n, t in self.times.items()}
+
+
+def run_ours(args):
+    import torch
+
+    from w8a8_quantized_gemm_b200 import sq
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    use_dist = _init_pg(ws, local)
+    dev = f"cuda:{local}"
+    hbm, bf16, bf16_sus, peak_kind = _peaks()
+    int8_peak = 2.0 * bf16  # nominal dense int8 : bf16 ratio of 2 (4.5 / 2.25 PFLOP/s)
+
+    p = wl.llama7b_mlp_up()
+    M, N, K = p.M, p.N, p.K
+    path = Path(p, dev, N_SETS)
+
+    for i in range(args.warmup):
+        path.step(i)
+    sq.sq_sync_status()
+    k_o = int(path.cnt.item())
+    ops_step = 2.0 * M * N * K * 2 + 2.0 * M * N * k_o
+
+    # ---------------------------------------------------------------- timed region
+    records = []
+    torch.cuda.synchronize()
+    _barrier(use_dist, local)
+    torch.cuda.synchronize()
+    launches0 = sq.sq_kernel_launch_count()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t_start.record()
+        for i in range(args.steps):
+            path.step(i, records)
+        t_end.record()
+        torch.cuda.synchronize()
+    launches = sq.sq_kernel_launch_count() - launches0
+    _barrier(use_dist, local)
+    torch.cuda.synchronize()
+    ms_total = t_start.elapsed_time(t_end)
+    ms_total = _max_over_ranks(ms_total, use_dist, local)
+    sq.sq_sync_status()
+    per_kernel = path.collect(records)
+
+    ms_step = ms_total / args.steps
+    value = ops_step * ws * args.steps / (ms_total * 1e-3) / 1e12
+
+    # ---------------------------------------------------------------- kernel rooflines
+    gemm_ms = per_kernel["int8_gemm_dequant"]
+    gemm_tops = 2.0 * M * N * K / (gemm_ms * 1e-3) / 1e12
+    traffic = NCU_GEMM_TRAFFIC_BYTES if (NCU_GEMM_TRAFFIC_BYTES and GEMM_SRC_SHA == _gemm_src_sha()) else None
+    roofline = {"kernel": "w8a8_gemm_kernel (sq_int8_gemm_dequant)", "bound": "tensor",
+                "achieved": round(gemm_tops, 1), "peak": round(int8_peak, 1), "unit": "TFLOP/s",
+                "frac": round(gemm_tops / int8_peak, 4), "traffic": traffic,
+                "peak_note": f"int8 dense = 2 x {peak_kind} bf16 burst {bf16} TFLOP/s (nominal int8:bf16 = 2); "
+                             f"vs 4500 datasheet: {gemm_tops / 4500.0:.3f}"}
+    hbm_bytes = {
+        "act_channel_absmax": 2.0 * M * K + 4 * K,
+        "smooth_scale": 2.0 * N * K + 12 * K,
+        "smooth_quant_weight": 3.0 * N * K + 4 * N + 4 * K,
+        "quant_act_per_token": 3.0 * M * K + 4 * M + 4 * K,
+        "quant_weight_unsmoothed": 3.0 * N * K + 4 * N,
+    }
+    kernels = {}
+    for n, t in per_kernel.items():
+        ent = {"us": round(t * 1e3, 2)}
+        if n in hbm_bytes:
+            gbs = hbm_bytes[n] / (t * 1e-3) / 1e9
+            ent.update({"GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)})
+        elif n == "int8_gemm_dequant":
+            ent.update({"TOPS": round(gemm_tops, 1), "frac_int8_peak": round(gemm_tops / int8_peak, 4)})
+        else:
+            tops = (2.0 * M * N * K + 2.0 * M * N * k_o) / (t * 1e-3) / 1e12
+            ent.update({"TOPS": round(tops, 1), "frac_int8_peak": round(tops / int8_peak, 4), "k_outliers": k_o})
+        kernels[n] = ent
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    e2e = run_e2e(path, p, args, ops_step, use_dist, local, ws)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded numpy PCG64, bf16)",
+        "config": {"workload": f"llama7b_mlp_up X[{M},{K}] W[{N},{K}]: SmoothQuant W8A8 linear (alpha {ALPHA}, "
+                               f"per-token act, per-channel weight) + LLM.int8 linear (threshold {THRESHOLD})",
+                   "M": M, "N": N, "K": K, "outlier_columns": k_o, "ops_per_step": ops_step,
+                   "l2": f"{N_SETS} rotating input sets ({N_SETS * (2 * M * K + 2 * N * K) / 1e6:.0f} MB) > L2",
+                   "parallelism": f"replica x{ws}"},
+        "roofline": roofline, "kernels": kernels, "gpu_launches": int(launches),
+        "clocks": clk.summary(), "e2e": e2e, "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16, "kind": peak_kind},
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(p, args.cpu_budget)
+    if use_dist:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(path, p, args, ops_step, use_dist, local, ws):
+    """Same step through the C ABI with the inputs in pinned HOST memory: H2D of X and W,
+    the step, D2H of both outputs, all inside the timed region."""
+    import torch
+    steps = max(3, min(args.steps, args.e2e_steps))
+    hX = torch.from_numpy(np.ascontiguousarray(p.X).view(np.int16)).view(torch.bfloat16).pin_memory()
+    hW = torch.from_numpy(np.ascontiguousarray(p.W).view(np.int16)).view(torch.bfloat16).pin_memory()
+    hY = torch.empty(path.Y.shape, dtype=torch.bfloat16).pin_memory()
+    hY2 = torch.empty(path.Y2.shape, dtype=torch.bfloat16).pin_memory()
+
+    def one(i):
+        k = i % len(path.X)
+        path.X[k].copy_(hX, non_blocking=True)
+        path.W[k].copy_(hW, non_blocking=True)
+        path.step(k)
+        hY.copy_(path.Y, non_blocking=True)
+        hY2.copy_(path.Y2, non_blocking=True)
+
+    for i in range(2):
+        one(i)
+    torch.cuda.synchronize()
+    _barrier(use_dist, local)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(steps):
+        one(i)
+    b.record()
+    torch.cuda.synchronize()
+    ms = _max_over_ranks(a.elapsed_time(b), use_dist, local)
+    bi = hX.numel() * 2 + hW.numel() * 2
+    bo = hY.numel() * 2 + hY2.numel() * 2
+    return {"value": round(ops_step * ws * steps / (ms * 1e-3) / 1e12, 3), "unit": "TOPS",
+            "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "steps": steps,
+            "ms_per_step": round(ms / steps, 3)}
+
+
+# ----------------------------------------------------------------------------- oracle on the host
+def _oracle_step(p, rows, oracle):
+    """The whole step on the host oracle, for a sample of token rows with the full weight."""
+    amax = oracle.act_channel_absmax(p.X)
+    s, inv_s = oracle.smooth_scale(amax, p.W, ALPHA)
+    Wq, e = oracle.smooth_quant_weight(p.W, s, oracle.PER_CHANNEL)
+    xq, d = oracle.quant_act_per_token(p.X[rows], inv_s)
+    oracle.dequant(oracle.int8_gemm(xq, Wq), d, e, None)
+    mask, idx, _ = oracle.outlier_columns(amax, THRESHOLD)
+    Wq0, e0 = oracle.smooth_quant_weight(p.W, None, oracle.PER_CHANNEL)
+    xq0, d0 = oracle.quant_act_per_token(p.X[rows], None, mask)
+    o = oracle.outlier_product(p.X[rows], p.W, idx)
+    oracle.dequant(oracle.int8_gemm(xq0, Wq0), d0, e0, None, o)
+    return len(idx)
+
+
+def _sample_rows(M, R):
+    return np.sort(np.random.default_rng(7).choice(M, R, replace=False))
+
+
+def cpu_baseline(p, budget_s):
+    import oracle
+    R = 8
+    rows = _sample_rows(p.M, R)
+    t0 = time.perf_counter()
+    k_o = _oracle_step(p, rows, oracle)
+    t1 = time.perf_counter()
+    # grow the sample towards the time budget (the per-row GEMM dominates)
+    R2 = int(min(p.M, max(R, R * budget_s / max(t1 - t0, 1e-3) * 0.8)))
+    if R2 > R:
+        rows = _sample_rows(p.M, R2)
+        t0 = time.perf_counter()
+        k_o = _oracle_step(p, rows, oracle)
+        t1 = time.perf_counter()
+        R = R2
+    ops = 2.0 * R * p.N * p.K * 2 + 2.0 * R * p.N * k_o
+    return {"value": round(ops / (t1 - t0) / 1e12, 6), "unit": "TOPS", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": round(t1 - t0, 3),
+            "sample": f"whole step (calibration, smoothing, both weight quantizations on the full W) with "
+                      f"{R} of {p.M} token rows through both GEMMs"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step is the whole path on a row sample."""
+    ws, rank, local = _dist()
+    if rank != 0:
+        return
+    import oracle
+    p = wl.llama7b_mlp_up()
+    R = args.ref_rows
+    rows = _sample_rows(p.M, R)
+    for _ in range(args.warmup):
+        k_o = _oracle_step(p, rows, oracle)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        k_o = _oracle_step(p, rows, oracle)
+    t1 = time.perf_counter()
+    ops = (2.0 * R * p.N * p.K * 2 + 2.0 * R * p.N * k_o) * args.steps
+    value = ops / (t1 - t0) / 1e12
+    sample = f"whole step with {R} of {p.M} token rows through both GEMMs (full-weight preparation)"
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round((t1 - t0) * 1e3 / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "data": "synthetic (seeded numpy PCG64, bf16)",
+            "config": {"workload": f"llama7b_mlp_up X[{p.M},{p.K}] W[{p.N},{p.K}] (row sample {R})",
+                       "M": p.M, "N": p.N, "K": p.K},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=4, help="token rows per reference-arm step")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -184,6 +184,10 @@ SQ_API sq_status sq_sync_status(sq_stream_t stream);
 /* Library version string and the compute capability it was built for ("sm_100a"). */
 SQ_API const char* sq_version(void);
 
+/* Number of kernels this library has launched in this process (all devices, all threads),
+ * for checking which work ran on the GPU. */
+SQ_API uint64_t sq_kernel_launch_count(void);
+
 /* Test hook for the failure path (no counterpart on the pages). Arms the NEXT
  * sq_int8_gemm_dequant call made on the calling thread: its device-side waits give up after
  * wait_limit_ns nanoseconds (0 = the default of 2 s) and, when fault == 1, its TMA producer

@@ -1,0 +1,90 @@
+"""The C ABI without a GPU: the library loads, exports exactly what include/sq.h
+declares, sizes workspaces, and rejects bad arguments before launching anything
+(validation never touches the device, so these calls are safe on a CPU-only host)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from w8a8_quantized_gemm_b200 import sq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "sq.h")).read()
+    return re.findall(r"SQ_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_header_symbols_exported():
+    names = _declared()
+    assert set(names) >= {"sq_act_channel_absmax", "sq_smooth_scale", "sq_smooth_quant_weight",
+                          "sq_quant_act_per_token", "sq_int8_gemm_dequant", "llmint8_decomposed_linear",
+                          "sq_workspace_size", "sq_last_error", "sq_sync_status"}
+    lib = C.CDLL(sq.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_only_declared_symbols_exported():
+    out = os.popen(f"nm -D --defined-only {sq.LIB_PATH}").read().split("\n")
+    exported = {l.split()[-1] for l in out if " T " in l}
+    assert exported == set(_declared())
+
+
+def test_version():
+    assert "sm_100a" in sq.sq_version()
+
+
+def test_workspace_sizes():
+    assert sq.sq_workspace_size(sq.SQ_OP_SMOOTH_QUANT_WEIGHT, 0, 100, 64) >= 4
+    M, N, K = 2048, 11008, 4096
+    ws = sq.sq_workspace_size(sq.SQ_OP_LLMINT8, M, N, K)
+    # int8 activations + gathered bf16 outlier operands (worst case: every column)
+    assert ws >= M * K + 2 * (M + N) * K
+    assert sq.sq_workspace_size(99, M, N, K) == 0
+
+
+FAKE = 1 << 20  # a 16-byte-aligned non-null address; never dereferenced on these paths
+
+
+def _raw():
+    return sq.lib()
+
+
+@pytest.mark.parametrize("M,K,ld,code", [(0, 64, 64, sq.SQ_ERR_INVALID), (4, 20, 20, sq.SQ_ERR_INVALID),
+                                         (4, 64, 32, sq.SQ_ERR_INVALID), (4, 64, 68, sq.SQ_ERR_ALIGN),
+                                         (4, 65552, 65552, sq.SQ_ERR_INVALID)])
+def test_absmax_validation(M, K, ld, code):
+    assert _raw().sq_act_channel_absmax(FAKE, M, K, ld, FAKE, 0, None) == code
+    assert sq.sq_last_error() != ""
+
+
+def test_null_and_alignment_rejected():
+    L = _raw()
+    assert L.sq_quant_act_per_token(None, 4, 64, 64, None, FAKE, FAKE, None) == sq.SQ_ERR_INVALID
+    assert L.sq_quant_act_per_token(FAKE + 8, 4, 64, 64, None, FAKE, FAKE, None) == sq.SQ_ERR_ALIGN
+    assert L.sq_smooth_scale(FAKE, FAKE, 8, 64, 64, C.c_float(1.5), FAKE, FAKE + 256, None) == sq.SQ_ERR_INVALID
+    assert L.sq_smooth_scale(FAKE, FAKE, 8, 64, 64, C.c_float(0.5), FAKE, FAKE, None) == sq.SQ_ERR_INVALID
+
+
+def test_gemm_validation():
+    L = _raw()
+    # N not a multiple of 8
+    assert L.sq_int8_gemm_dequant(FAKE, FAKE, FAKE, FAKE, 1, None, FAKE, 16, 12, 64, None, None, 0, None) \
+        == sq.SQ_ERR_INVALID
+    # bad granularity
+    assert L.sq_int8_gemm_dequant(FAKE, FAKE, FAKE, FAKE, 7, None, FAKE, 16, 16, 64, None, None, 0, None) \
+        == sq.SQ_ERR_INVALID
+    # per-tensor weight quantization without workspace
+    assert L.sq_smooth_quant_weight(FAKE, 8, 64, 64, None, 0, FAKE, FAKE, None, 0, None) == sq.SQ_ERR_WORKSPACE
+
+
+def test_llmint8_validation():
+    L = _raw()
+    need = sq.sq_workspace_size(sq.SQ_OP_LLMINT8, 16, 16, 64)
+    assert L.llmint8_decomposed_linear(FAKE, FAKE, FAKE, FAKE, C.c_float(6.0), None, FAKE, 16, 16, 64, None, None,
+                                       None, FAKE, need - 1, None) == sq.SQ_ERR_WORKSPACE
+    assert L.llmint8_decomposed_linear(FAKE, FAKE, FAKE, FAKE, C.c_float(float("nan")), None, FAKE, 16, 16, 64,
+                                       None, None, None, FAKE, need, None) == sq.SQ_ERR_INVALID

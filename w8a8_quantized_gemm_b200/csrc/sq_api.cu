@@ -4,6 +4,7 @@
 #include "sq.h"
 #include "sq_internal.h"
 
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -25,6 +26,11 @@ unsigned int* device_status_word() {
   }
   return addr[dev];
 }
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 }  // namespace sq
 
@@ -331,6 +337,8 @@ sq_status sq_sync_status(sq_stream_t stream) {
 }
 
 const char* sq_version(void) { return "libsq 0.1 sm_100a"; }
+
+uint64_t sq_kernel_launch_count(void) { return sq::g_launches.load(); }
 
 void sq_debug_arm_fault(int fault, uint64_t wait_limit_ns) {
   g_arm_fault = fault;

@@ -436,6 +436,7 @@ cudaError_t run(const GemmArgs& a, cudaStream_t stream, const char** why) {
   p.fault = a.fault;
   const int tiles = p.num_m_tiles * p.num_n_tiles;
   const int grid = std::min(tiles, num_sms());
+  note_launch();
   w8a8_gemm_kernel<BN, OUTLIERS><<<grid, kThreads, C::kSmemBytes, stream>>>(tmA, tmB, tmXo, tmWo, p);
   return cudaGetLastError();
 }

@@ -20,6 +20,9 @@ constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s per wait
 // Device address of the error word of the current device.
 unsigned int* device_status_word();
 
+// Host-side count of kernels this library has launched (diagnostics).
+void note_launch();
+
 // ---- reductions (sq_reduce.cu)
 // Column absmax of a bf16 [rows, K] matrix into amax (fp32 [K], stored as ordered bits).
 // With accumulate == 0 the output is reset first.

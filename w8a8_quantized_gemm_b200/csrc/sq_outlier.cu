@@ -81,6 +81,7 @@ __global__ void gather_columns_kernel(const uint16_t* __restrict__ src, int64_t 
 cudaError_t launch_outlier_mask(const float* amax, int64_t K, float threshold, uint32_t* mask, int32_t* prefix,
                                 int32_t* idx, int32_t* count, uint32_t* mask_out, int32_t* count_out,
                                 cudaStream_t stream) {
+  note_launch();
   outlier_mask_kernel<<<1, kMaskThreads, 0, stream>>>(amax, K, threshold, mask, prefix, idx, count, mask_out,
                                                        count_out);
   return cudaGetLastError();
@@ -91,6 +92,7 @@ cudaError_t launch_gather_columns(const uint16_t* src, int64_t rows, int64_t ld,
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  note_launch();
   gather_columns_kernel<<<sms * 4, 256, 0, stream>>>(src, rows, ld, idx, count, dst, ld_dst);
   return cudaGetLastError();
 }

@@ -203,6 +203,7 @@ cudaError_t launch_t(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, c
   constexpr int kThreads = TPR > kCta ? TPR : kCta;
   constexpr int kGroups = kThreads / TPR;
   const int64_t blocks = (rows + kGroups - 1) / kGroups;
+  note_launch();
   quant_rows_kernel<TPR, CHUNKS, TWO_PASS, OUTLIERS, MODE>
       <<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(src, rows, K, ld, vec, ov, q, scale, gmax);
   return cudaGetLastError();

@@ -117,6 +117,7 @@ cudaError_t launch_col_absmax(const uint16_t* src, int64_t rows, int64_t K, int6
     rows_per_cta = (rows + row_blocks - 1) / row_blocks;
   }
   dim3 grid(static_cast<unsigned>(col_blocks), static_cast<unsigned>(row_blocks));
+  note_launch();
   col_absmax_kernel<<<grid, kColWarps * 32, 0, stream>>>(src, rows, K, ld, rows_per_cta,
                                                          reinterpret_cast<unsigned int*>(amax));
   return cudaGetLastError();
@@ -126,6 +127,7 @@ cudaError_t launch_smooth_factors(const float* act_amax, float* s_inout, float* 
                                   cudaStream_t stream) {
   const int threads = 256;
   const int64_t blocks = (K + threads - 1) / threads;
+  note_launch();
   smooth_factors_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(act_amax, s_inout, inv_s, K, alpha);
   return cudaGetLastError();
 }

@@ -38,6 +38,7 @@ _SIGS = {
     "sq_sync_status": ([_p], _i32),
     "sq_version": ([], C.c_char_p),
     "sq_debug_arm_fault": ([_i32, C.c_uint64], None),
+    "sq_kernel_launch_count": ([], C.c_uint64),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -155,6 +156,7 @@ def sq_int8_gemm_dequant(Xq, Wq, x_scale, w_scale, w_gran: int, bias, Y, acc_out
 
 def llmint8_decomposed_linear(X, W, Wq, w_scale, threshold: float, bias, Y, mask_out=None, n_outliers_out=None,
                               acc_out=None, ws=None, stream=None):
+    """mask_out is passed as a torch.int32 tensor of ceil(K/32) words (same bits as uint32)."""
     torch = _torch()
     M, K = X.shape
     N = W.shape[0]
@@ -174,6 +176,10 @@ def sq_workspace_size(op: int, M: int, N: int, K: int) -> int:
 
 def sq_sync_status(stream=None):
     _check(_lib.sq_sync_status(_stream(stream)))
+
+
+def sq_kernel_launch_count() -> int:
+    return int(_lib.sq_kernel_launch_count())
 
 
 def sq_debug_arm_fault(fault: int, wait_limit_ns: int = 0):

@@ -36,10 +36,14 @@ _ROLES = ("x", "cols", "mag", "w", "bias", "calib")
 
 
 def f32_to_bf16_bits(a) -> np.ndarray:
-    """Pack float32 values as bf16 bit patterns, round-to-nearest-even (format conversion only)."""
-    u = np.ascontiguousarray(np.asarray(a, dtype=np.float32)).view(np.uint32).astype(np.uint64)
-    lsb = (u >> np.uint64(16)) & np.uint64(1)
-    return ((u + np.uint64(0x7FFF) + lsb) >> np.uint64(16)).astype(np.uint16)
+    """Pack finite float32 values as bf16 bit patterns, round-to-nearest-even (format conversion only)."""
+    u = np.array(np.asarray(a, dtype=np.float32), copy=True, order="C").view(np.uint32)
+    lsb = u >> np.uint32(16)
+    lsb &= np.uint32(1)
+    u += np.uint32(0x7FFF)
+    u += lsb
+    u >>= np.uint32(16)
+    return u.astype(np.uint16)
 
 
 def bf16_bits_to_f32(b) -> np.ndarray:
@@ -81,7 +85,9 @@ class Problem:
 
 
 def _normal(rng, shape, sigma):
-    return rng.standard_normal(shape, dtype=np.float32) * np.float32(sigma)
+    x = rng.standard_normal(shape, dtype=np.float32)
+    x *= np.float32(sigma)
+    return x
 
 
 def _pick_cols(rng, K, n):

@@ -168,6 +168,27 @@ SQ_API sq_status llmint8_decomposed_linear(const void* X_bf16, const void* W_bf1
                                     int32_t* n_outliers_out, int32_t* acc_out, void* ws, size_t ws_bytes,
                                     sq_stream_t stream);
 
+/*
+ * Variant of sq_smooth_quant_weight that allocates nothing and takes no workspace, for
+ * callers that cannot allocate device memory: components running inside a host engine,
+ * server or plugin interface that owns the whole device-memory plan and passes them only
+ * the tensors of the current call, and services that fix their memory footprint at
+ * start-up. It has no counterpart on the pages; the quantization it performs is exactly
+ * that of sq_smooth_quant_weight (same arguments minus ws/ws_bytes, same results).
+ * Scratch: a 256-byte static device array inside the library (the per-tensor form keeps its
+ * global maximum there; the per-channel form needs none). Every GPU that loads the library
+ * holds those bytes until the process exits. A shape that would need more scratch than the
+ * array holds is rejected with SQ_ERR_WORKSPACE and a message naming both sizes.
+ * Set-up: the first call on each device looks the array's device address up (with that
+ * device current); make that first call before any stream capture.
+ * Concurrency: all calls share the array and it keeps the last call's contents; each
+ * per-tensor call resets the maximum it needs before use, but calls that overlap on the GPU
+ * (different streams, or several host threads) race on it and must be serialised.
+ */
+SQ_API sq_status sq_smooth_quant_weight_noalloc(const void* W_bf16, int64_t N, int64_t K, int64_t ldw,
+                                                const float* s, sq_gran gran, int8_t* Wq, float* w_scale,
+                                                sq_stream_t stream);
+
 /* Bytes of scratch an operation needs for the given shape (0 if none). Returns 0 for an
  * unknown op; never fails otherwise. */
 SQ_API size_t sq_workspace_size(int op, int64_t M, int64_t N, int64_t K);

@@ -51,6 +51,15 @@ sq_status fail(sq_status st, const char* fmt, ...) {
   return st;
 }
 
+}  // namespace
+
+int sq::record_error(int st, const char* msg) {
+  g_last_error = msg;
+  return st;
+}
+
+namespace {
+
 sq_status cuda_fail(cudaError_t e, const char* what) {
   return fail(SQ_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }

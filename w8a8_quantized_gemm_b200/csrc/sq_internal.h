@@ -23,6 +23,9 @@ unsigned int* device_status_word();
 // Host-side count of kernels this library has launched (diagnostics).
 void note_launch();
 
+// Records the message returned by sq_last_error() on this thread; returns st.
+int record_error(int st, const char* msg);
+
 // ---- reductions (sq_reduce.cu)
 // Column absmax of a bf16 [rows, K] matrix into amax (fp32 [K], stored as ordered bits).
 // With accumulate == 0 the output is reset first.

@@ -33,6 +33,7 @@ _SIGS = {
     "sq_quant_act_per_token": ([_p, _i64, _i64, _i64, _p, _p, _p, _p], _i32),
     "sq_int8_gemm_dequant": ([_p, _p, _p, _p, _i32, _p, _p, _i64, _i64, _i64, _p, _p, _sz, _p], _i32),
     "llmint8_decomposed_linear": ([_p, _p, _p, _p, _f32, _p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _sz, _p], _i32),
+    "sq_smooth_quant_weight_noalloc": ([_p, _i64, _i64, _i64, _p, _i32, _p, _p, _p], _i32),
     "sq_workspace_size": ([_i32, _i64, _i64, _i64], _sz),
     "sq_last_error": ([], C.c_char_p),
     "sq_sync_status": ([_p], _i32),
@@ -130,6 +131,18 @@ def sq_smooth_quant_weight(W, s, gran: int, Wq, w_scale, ws=None, stream=None):
     _check(_lib.sq_smooth_quant_weight(_ptr(W, torch.bfloat16, "W", True), N, K, W.stride(0),
                                        _ptr(s, torch.float32, "s"), int(gran), _ptr(Wq, torch.int8, "Wq"),
                                        _ptr(w_scale, torch.float32, "w_scale"), wsp, wsb, _stream(stream)))
+    return Wq, w_scale
+
+
+def sq_smooth_quant_weight_noalloc(W, s, gran: int, Wq, w_scale, stream=None):
+    """sq_smooth_quant_weight without a workspace (scratch lives in the library), for
+    callers that cannot allocate device memory; calls overlapping on the GPU must not run
+    concurrently."""
+    torch = _torch()
+    N, K = W.shape
+    _check(_lib.sq_smooth_quant_weight_noalloc(_ptr(W, torch.bfloat16, "W", True), N, K, W.stride(0),
+                                               _ptr(s, torch.float32, "s"), int(gran), _ptr(Wq, torch.int8, "Wq"),
+                                               _ptr(w_scale, torch.float32, "w_scale"), _stream(stream)))
     return Wq, w_scale
 
 

@@ -194,13 +194,13 @@ class Path:
         self.times = {n: 0.0 for n in self.names}
         self.ev_pool = []
 
-    def step(self, i, record=None):
+    def step(self, i, record=None, external=False):
         sq, X, W = self.sq, self.X[i % len(self.X)], self.W[i % len(self.W)]
         ev = []
 
         def mark():
             if record is not None:
-                e = self.torch.cuda.Event(enable_timing=True)
+                e = self.torch.cuda.Event(enable_timing=True, external=external)
                 e.record()
                 ev.append(e)
 
@@ -253,26 +253,53 @@ def run_ours(args):
     ops_step = 2.0 * M * N * K * 2 + 2.0 * M * N * k_o
 
     # ---------------------------------------------------------------- timed region
+    # The K timed steps are captured once as one CUDA graph (launch overhead out of the way,
+    # as a serving loop would run them), with timing events between the operations of every
+    # step; the graph is replayed once untimed and once timed.
     records = []
+    mode = "cuda_graph"
+    stream = torch.cuda.Stream()
+    graph = None
+    launches0 = sq.sq_kernel_launch_count()
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(args.steps):
+                path.step(i, records, external=True)
+        launches = sq.sq_kernel_launch_count() - launches0
+        with torch.cuda.stream(stream):
+            graph.replay()
+        torch.cuda.synchronize()
+    except Exception as exc:  # capture unsupported here: time the same steps eagerly
+        mode = f"eager ({type(exc).__name__})"
+        graph, records = None, []
+        torch.cuda.synchronize()
     torch.cuda.synchronize()
     _barrier(use_dist, local)
     torch.cuda.synchronize()
-    launches0 = sq.sq_kernel_launch_count()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
-        t_start.record()
-        for i in range(args.steps):
-            path.step(i, records)
-        t_end.record()
+        with torch.cuda.stream(stream):
+            if graph is not None:
+                t_start.record()
+                graph.replay()
+                t_end.record()
+            else:
+                launches0 = sq.sq_kernel_launch_count()
+                t_start.record()
+                for i in range(args.steps):
+                    path.step(i, records)
+                t_end.record()
+                launches = sq.sq_kernel_launch_count() - launches0
         torch.cuda.synchronize()
-    launches = sq.sq_kernel_launch_count() - launches0
     _barrier(use_dist, local)
     torch.cuda.synchronize()
     ms_total = t_start.elapsed_time(t_end)
     ms_total = _max_over_ranks(ms_total, use_dist, local)
     sq.sq_sync_status()
     per_kernel = path.collect(records)
+    del graph
 
     ms_step = ms_total / args.steps
     value = ops_step * ws * args.steps / (ms_total * 1e-3) / 1e12
@@ -318,7 +345,7 @@ def run_ours(args):
                    "M": M, "N": N, "K": K, "outlier_columns": k_o, "ops_per_step": ops_step,
                    "l2": f"{N_SETS} rotating input sets ({N_SETS * (2 * M * K + 2 * N * K) / 1e6:.0f} MB) > L2",
                    "parallelism": f"replica x{ws}"},
-        "roofline": roofline, "kernels": kernels, "gpu_launches": int(launches),
+        "roofline": roofline, "kernels": kernels, "gpu_launches": int(launches), "launch_mode": mode,
         "clocks": clk.summary(), "e2e": e2e, "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16, "kind": peak_kind},
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -367,70 +394,83 @@ def run_e2e(path, p, args, ops_step, use_dist, local, ws):
 
 
 # ----------------------------------------------------------------------------- oracle on the host
-def _oracle_step(p, rows, oracle):
-    """The whole step on the host oracle, for a sample of token rows with the full weight."""
-    amax = oracle.act_channel_absmax(p.X)
-    s, inv_s = oracle.smooth_scale(amax, p.W, ALPHA)
-    Wq, e = oracle.smooth_quant_weight(p.W, s, oracle.PER_CHANNEL)
-    xq, d = oracle.quant_act_per_token(p.X[rows], inv_s)
+def _sample(p, R, Nr):
+    """A sub-problem of the workload: R token rows of X and Nr output rows of W (seeded)."""
+    rng = np.random.default_rng(7)
+    rows = np.sort(rng.choice(p.M, R, replace=False)) if R < p.M else np.arange(p.M)
+    wrows = np.sort(rng.choice(p.N, Nr, replace=False)) if Nr < p.N else np.arange(p.N)
+    return np.ascontiguousarray(p.X[rows]), np.ascontiguousarray(p.W[wrows])
+
+
+def _oracle_step(X, W, oracle):
+    """The whole step on the host oracle for the linear X [R,K] x W [Nr,K]: both linears,
+    calibration and weight preparation included. Returns (tensor ops, K_o)."""
+    amax = oracle.act_channel_absmax(X)
+    s, inv_s = oracle.smooth_scale(amax, W, ALPHA)
+    Wq, e = oracle.smooth_quant_weight(W, s, oracle.PER_CHANNEL)
+    xq, d = oracle.quant_act_per_token(X, inv_s)
     oracle.dequant(oracle.int8_gemm(xq, Wq), d, e, None)
-    mask, idx, _ = oracle.outlier_columns(amax, THRESHOLD)
-    Wq0, e0 = oracle.smooth_quant_weight(p.W, None, oracle.PER_CHANNEL)
-    xq0, d0 = oracle.quant_act_per_token(p.X[rows], None, mask)
-    o = oracle.outlier_product(p.X[rows], p.W, idx)
+    mask, idx, k_o = oracle.outlier_columns(amax, THRESHOLD)
+    Wq0, e0 = oracle.smooth_quant_weight(W, None, oracle.PER_CHANNEL)
+    xq0, d0 = oracle.quant_act_per_token(X, None, mask)
+    o = oracle.outlier_product(X, W, idx)
     oracle.dequant(oracle.int8_gemm(xq0, Wq0), d0, e0, None, o)
-    return len(idx)
-
-
-def _sample_rows(M, R):
-    return np.sort(np.random.default_rng(7).choice(M, R, replace=False))
+    R, K = X.shape
+    Nr = W.shape[0]
+    return 2.0 * R * Nr * K * 2 + 2.0 * R * Nr * k_o, k_o
 
 
 def cpu_baseline(p, budget_s):
+    """The oracle, as it stands, on the whole step of the workload (all rows), repeated until
+    about `budget_s` seconds of host work (at most 3 repetitions)."""
     import oracle
-    R = 8
-    rows = _sample_rows(p.M, R)
-    t0 = time.perf_counter()
-    k_o = _oracle_step(p, rows, oracle)
-    t1 = time.perf_counter()
-    # grow the sample towards the time budget (the per-row GEMM dominates)
-    R2 = int(min(p.M, max(R, R * budget_s / max(t1 - t0, 1e-3) * 0.8)))
-    if R2 > R:
-        rows = _sample_rows(p.M, R2)
+    X, W = p.X, p.W
+    reps, ops, t = 0, 0.0, 0.0
+    while reps < 3 and (reps == 0 or t < budget_s):
         t0 = time.perf_counter()
-        k_o = _oracle_step(p, rows, oracle)
-        t1 = time.perf_counter()
-        R = R2
-    ops = 2.0 * R * p.N * p.K * 2 + 2.0 * R * p.N * k_o
-    return {"value": round(ops / (t1 - t0) / 1e12, 6), "unit": "TOPS", "cores": oracle.num_threads(),
-            "kind": "oracle", "seconds": round(t1 - t0, 3),
-            "sample": f"whole step (calibration, smoothing, both weight quantizations on the full W) with "
-                      f"{R} of {p.M} token rows through both GEMMs"}
+        o, _ = _oracle_step(X, W, oracle)
+        t += time.perf_counter() - t0
+        ops += o
+        reps += 1
+    return {"value": round(ops / t / 1e12, 6), "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
+            "seconds": round(t, 3),
+            "sample": f"the whole step on the full workload ({p.M} token rows, {p.N} output channels), {reps} run(s)"}
 
 
 def run_reference(args):
-    """The oracle as the reference arm: each step is the whole path on a row sample."""
+    """The oracle as the reference arm: each step is the whole path on a seeded sub-problem of
+    the workload (a subset of token rows and output channels, full K), sized so that the
+    --steps/--warmup run ends within a couple of minutes."""
     ws, rank, local = _dist()
     if rank != 0:
         return
     import oracle
     p = wl.llama7b_mlp_up()
-    R = args.ref_rows
-    rows = _sample_rows(p.M, R)
+    R = min(args.ref_rows, p.M)
+    Nr = min(1024, p.N)
+    X, W = _sample(p, R, Nr)
+    t0 = time.perf_counter()
+    _oracle_step(X, W, oracle)
+    t1 = time.perf_counter()
+    per_step_target = min(1.0, 120.0 / max(1, args.steps + args.warmup))
+    Nr = int(min(p.N, max(64, Nr * per_step_target / max(t1 - t0, 1e-4))))
+    X, W = _sample(p, R, Nr)
     for _ in range(args.warmup):
-        k_o = _oracle_step(p, rows, oracle)
+        _oracle_step(X, W, oracle)
+    ops = 0.0
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        k_o = _oracle_step(p, rows, oracle)
+        o, k_o = _oracle_step(X, W, oracle)
+        ops += o
     t1 = time.perf_counter()
-    ops = (2.0 * R * p.N * p.K * 2 + 2.0 * R * p.N * k_o) * args.steps
     value = ops / (t1 - t0) / 1e12
-    sample = f"whole step with {R} of {p.M} token rows through both GEMMs (full-weight preparation)"
+    sample = (f"whole step (calibration, smoothing, both weight quantizations, both linears) on {R} of {p.M} "
+              f"token rows x {Nr} of {p.N} output channels, K={p.K}")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round((t1 - t0) * 1e3 / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
             "data": "synthetic (seeded numpy PCG64, bf16)",
-            "config": {"workload": f"llama7b_mlp_up X[{p.M},{p.K}] W[{p.N},{p.K}] (row sample {R})",
+            "config": {"workload": f"llama7b_mlp_up X[{p.M},{p.K}] W[{p.N},{p.K}] (sub-problem {R}x{Nr})",
                        "M": p.M, "N": p.N, "K": p.K},
             "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": sample},
@@ -441,13 +481,13 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-rows", type=int, default=4, help="token rows per reference-arm step")
+    ap.add_argument("--ref-rows", type=int, default=64, help="token rows per reference-arm step")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

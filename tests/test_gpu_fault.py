@@ -25,11 +25,12 @@ def test_withheld_stage_times_out_and_context_survives():
     acc = empty((M, N), torch.int32)
     sq.sq_sync_status()  # clean slate
     sq.sq_debug_arm_fault(1, 50_000_000)  # 50 ms per wait
-    sq.sq_int8_gemm_dequant(*args, sq.SQ_PER_CHANNEL, None, Y, acc)
+    sq.sq_int8_gemm_dequant(*args, sq.SQ_PER_CHANNEL, None, Y, acc, sq.workspace(sq.SQ_OP_INT8_GEMM_DEQUANT, M, N, K))
     with pytest.raises(sq.SqError) as ei:
         sq.sq_sync_status()
     assert ei.value.status == sq.SQ_ERR_TIMEOUT
-    # the status word was cleared and the context still works
-    sq.sq_int8_gemm_dequant(*args, sq.SQ_PER_CHANNEL, None, Y, acc)
+    # the status word was cleared and the context still works (with a fresh zeroed workspace:
+    # an aborted call may leave split-K arrival counters behind)
+    sq.sq_int8_gemm_dequant(*args, sq.SQ_PER_CHANNEL, None, Y, acc, sq.workspace(sq.SQ_OP_INT8_GEMM_DEQUANT, M, N, K))
     sq.sq_sync_status()
     assert np.array_equal(host(acc), oracle.int8_gemm(xq, wq))

@@ -28,8 +28,9 @@ def _gemm_direct(xq, wq, d, e, gran, bias_bits):
 
 # shapes: single tile, ragged in every dimension, K below one k-block, several tiles for the
 # BN = 64 / 128 / 256 variants (the variant depends on the tile count versus the SM count)
+# (128,128,4096), (257,1000,528), (3,200,1040) and (64,4096,4096) split K over int32 partials
 GEMM_SHAPES = [(1, 8, 16), (16, 256, 256), (5, 24, 48), (130, 72, 144), (200, 264, 208), (128, 128, 4096),
-               (257, 1000, 528), (1024, 2048, 1024), (2304, 2120, 720)]
+               (257, 1000, 528), (3, 200, 1040), (64, 4096, 4096), (1024, 2048, 1024), (2304, 2120, 720)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
@@ -86,6 +87,31 @@ def test_smoothquant_path_ragged(M, N, K, gran):
         assert np.array_equal(g[k], o[k]), k
     assert np.array_equal(g["Y"], o["y_bf16"])
     assert_close_bf16(g["Y"], o["y_ref"], p.name)
+
+
+def test_split_k_workspace_reused_across_calls():
+    """The split-K arrival counters return to zero, so one workspace serves call after call."""
+    M, N, K = 16, 1024, 4096
+    assert sq.sq_workspace_size(sq.SQ_OP_INT8_GEMM_DEQUANT, M, N, K) > 0
+    rng = np.random.default_rng(11)
+    ws = sq.workspace(sq.SQ_OP_INT8_GEMM_DEQUANT, M, N, K)
+    d = np.full(M, 1e-2, np.float32)
+    e = np.full(N, 1e-3, np.float32)
+    dd, ee = torch.from_numpy(d).cuda(), torch.from_numpy(e).cuda()
+    for rep in range(3):
+        xq = rng.integers(-127, 128, size=(M, K), dtype=np.int8)
+        wq = rng.integers(-127, 128, size=(N, K), dtype=np.int8)
+        Y = empty((M, N), torch.bfloat16)
+        acc = empty((M, N), torch.int32)
+        sq.sq_int8_gemm_dequant(torch.from_numpy(xq).cuda(), torch.from_numpy(wq).cuda(), dd, ee, sq.SQ_PER_CHANNEL,
+                                None, Y, acc, ws)
+        sq.sq_sync_status()
+        oacc = oracle.int8_gemm(xq, wq)
+        assert np.array_equal(host(acc), oacc)
+        assert np.array_equal(host_bits(Y), oracle.dequant(oacc, d, e)[1])
+    n_t = (N + 63) // 64
+    ctr = ws[-((n_t * 8 * 4 + 255) // 256 * 256):].view(torch.int32)
+    assert int(ctr.abs().sum()) == 0
 
 
 def test_repeated_calls_are_deterministic():

@@ -34,19 +34,26 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 128;  // bytes of K per stage row: 128 int8 or 64 bf16
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kStageTileBytes = 32 * 32 * 2;  // one 32-row x 32-column bf16 output box
+constexpr int kEpiBufs = 2;                   // per epilogue warp
+constexpr int kEpiSmem = kEpiWarps * kEpiBufs * kStageTileBytes;
 
-template <int BN, bool OUTLIERS>
+template <int BN, bool OUTLIERS, int ACC_BUFS>
 struct Cfg {
   static constexpr int kStageA = kBM * kBK;
   static constexpr int kStageB = BN * kBK;
   static constexpr int kStageBytes = kStageA + kStageB;
-  static constexpr int kStages = (200 * 1024) / kStageBytes;
+  static constexpr int kStages = (192 * 1024) / kStageBytes;
   static constexpr int kAccCols = OUTLIERS ? 2 * BN : BN;  // per buffer: int32 acc (+ fp32 acc)
-  static constexpr int kTmemCols = 2 * kAccCols;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kTmemCols = ACC_BUFS * kAccCols;
+  static constexpr int kBarOffset = kStages * kStageBytes + kEpiSmem;
+  static constexpr int kSmemBytes = kBarOffset + 256 /*barriers*/ + 1024 /*alignment slack*/;
   static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
   static_assert(kStages >= 3, "pipeline depth");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+  static_assert(BN % 64 == 0, "two epilogue column halves of whole 32-column chunks");
 };
 
 struct Params {
@@ -54,10 +61,13 @@ struct Params {
   const float* w_scale;
   int w_per_channel;
   const uint16_t* bias;
-  uint16_t* Y;
   int32_t* acc_out;
   int64_t M, N;
   int num_m_tiles, num_n_tiles, num_kb;
+  int splits;          // K splits per output tile (1: no split)
+  int kb_per_split;    // k-blocks per split
+  int32_t* partials;   // [splits][M][N] int32 (splits > 1)
+  int32_t* counters;   // [m_tiles * n_tiles * kEpiWarps] arrival counters (splits > 1), zero between calls
   const int32_t* o_count;
   unsigned int* status;
   uint64_t wait_limit_ns;
@@ -90,21 +100,97 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return l | (h << 16);
 }
 
-template <int BN, bool OUTLIERS>
+// Per-warp column constants of a 32-column chunk, spread over the lanes: lane l holds the
+// weight scales of columns 4*(l%8)..4*(l%8)+3 of chunk l/8 (float4) and their 4 bf16 biases,
+// so a warp covers 4 chunks (128 columns). Loaded before the accumulator is ready.
+struct ColConsts {
+  float4 e;
+  uint2 b;
+};
+
+__device__ __forceinline__ ColConsts load_col_consts(const Params& p, int64_t n_half0, int lane, int chunks) {
+  ColConsts cc;
+  const int c = lane >> 3;
+  const int64_t n = n_half0 + c * 32 + (lane & 7) * 4;
+  const bool ok = c < chunks && n < p.N;
+  if (p.w_per_channel) {
+    cc.e = ok ? __ldg(reinterpret_cast<const float4*>(p.w_scale + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  } else {
+    const float e0 = __ldg(p.w_scale);
+    cc.e = make_float4(e0, e0, e0, e0);
+  }
+  cc.b = (p.bias != nullptr && ok) ? __ldg(reinterpret_cast<const uint2*>(p.bias + n)) : make_uint2(0u, 0u);
+  return cc;
+}
+
+// y[j] = (float(acc[j]) * d_m) * e[n0+j] for the 32 columns of chunk c.
+__device__ __forceinline__ void dequant32(const uint32_t (&acc)[32], float d_m, const ColConsts& cc, int c,
+                                          float (&y)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    const int src = c * 8 + j / 4;
+    const float e[4] = {__shfl_sync(0xffffffffu, cc.e.x, src), __shfl_sync(0xffffffffu, cc.e.y, src),
+                        __shfl_sync(0xffffffffu, cc.e.z, src), __shfl_sync(0xffffffffu, cc.e.w, src)};
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      y[j + u] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(acc[j + u])), d_m), e[u]);
+  }
+}
+
+// y[j] += bias[n0+j] (when there is a bias), then pack to bf16 pairs.
+__device__ __forceinline__ void bias_pack32(float (&y)[32], bool has_bias, const ColConsts& cc, int c,
+                                            uint32_t (&out)[16]) {
+  if (has_bias) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      const int src = c * 8 + j / 4;
+      const uint32_t b0 = __shfl_sync(0xffffffffu, cc.b.x, src);
+      const uint32_t b1 = __shfl_sync(0xffffffffu, cc.b.y, src);
+      y[j] = __fadd_rn(y[j], __uint_as_float(b0 << 16));
+      y[j + 1] = __fadd_rn(y[j + 1], __uint_as_float(b0 & 0xFFFF0000u));
+      y[j + 2] = __fadd_rn(y[j + 2], __uint_as_float(b1 << 16));
+      y[j + 3] = __fadd_rn(y[j + 3], __uint_as_float(b1 & 0xFFFF0000u));
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) out[j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
+}
+
+// One 32x32 bf16 box (this lane's row, 32 columns) through the warp's staging buffer to a
+// TMA store at (n0, row0).
+__device__ __forceinline__ void store_box(const uint32_t (&v)[16], uint8_t* stage_tiles, int& ebuf, int lane,
+                                          const CUtensorMap* tmY, int64_t n0, int64_t row0) {
+  // staging buffer `ebuf` was last read by the TMA store issued two boxes ago
+  if (lane == 0) bulk_wait_group_read<kEpiBufs - 1>();
+  __syncwarp();
+  uint4* st = reinterpret_cast<uint4*>(stage_tiles + ebuf * kStageTileBytes + lane * 64);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) st[j] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmY, stage_tiles + ebuf * kStageTileBytes, static_cast<int32_t>(n0), static_cast<int32_t>(row0));
+    bulk_commit_group();
+  }
+  ebuf ^= 1;
+}
+
+template <int BN, bool OUTLIERS, int ACC_BUFS>
 __global__ void __launch_bounds__(kThreads, 1)
 w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmXo, const __grid_constant__ CUtensorMap tmWo,
-                 const Params p) {
-  using C = Cfg<BN, OUTLIERS>;
+                 const __grid_constant__ CUtensorMap tmY, const Params p) {
+  using C = Cfg<BN, OUTLIERS, ACC_BUFS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint8_t* epi_base = smem + C::kStages * C::kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   uint64_t* full = bars;
   uint64_t* empty = bars + C::kStages;
   uint64_t* tmem_full = bars + 2 * C::kStages;
-  uint64_t* tmem_empty = tmem_full + 2;
-  uint64_t* teardown = tmem_empty + 2;
+  uint64_t* tmem_empty = tmem_full + ACC_BUFS;
+  uint64_t* teardown = tmem_empty + ACC_BUFS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const Abort ab{abort_flag};
@@ -117,9 +203,9 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < ACC_BUFS; ++b) {
       mbar_init(tmem_full + b, 1);
-      mbar_init(tmem_empty + b, 4);
+      mbar_init(tmem_empty + b, kEpiWarps);
     }
     mbar_init(teardown, 1);
     *abort_flag = 0;
@@ -127,6 +213,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     fence_proxy_async_smem();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmY);
     if (OUTLIERS) {
       tma_prefetch_desc(&tmXo);
       tma_prefetch_desc(&tmWo);
@@ -141,11 +228,16 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int num_tiles = p.num_m_tiles * p.num_n_tiles;
-  const int kb_i8 = p.num_kb;
+  // tiles: m fastest, then n, then the K split
+  const int mn_tiles = p.num_m_tiles * p.num_n_tiles;
+  const int num_tiles = mn_tiles * p.splits;
   int kb_o = 0;
   if constexpr (OUTLIERS) kb_o = (__ldg(p.o_count) + 63) / 64;
-  const int kb_total = kb_i8 + kb_o;
+  auto kb_range = [&](int tile, int& kb_begin, int& kb_i8_end) {
+    const int split = tile / mn_tiles;
+    kb_begin = split * p.kb_per_split;
+    kb_i8_end = min(p.num_kb, kb_begin + p.kb_per_split);
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -157,8 +249,11 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       bool withheld = false;
       for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
         const int m0 = (tile % p.num_m_tiles) * kBM;
-        const int n0 = (tile / p.num_m_tiles) * BN;
-        for (int kb = 0; kb < kb_total; ++kb) {
+        const int n0 = ((tile % mn_tiles) / p.num_m_tiles) * BN;
+        int kb0, kb_i8;
+        kb_range(tile, kb0, kb_i8);
+        const int kb_total = kb_i8 + kb_o;
+        for (int kb = kb0; kb < kb_total; ++kb) {
           if (!wait_or_abort(empty + stage, phase ^ 1, p.wait_limit_ns, abort_flag)) {
             if (!*abort_flag) ab.raise(p.status, kErrProducerWait);
             break;
@@ -203,8 +298,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       uint32_t phase = 0;
       int it = 0;
       for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, ++it) {
-        const int buf = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
+        const int buf = it % ACC_BUFS;
+        const uint32_t acc_phase = (it / ACC_BUFS) & 1;
         if (!wait_or_abort(tmem_empty + buf, acc_phase ^ 1, p.wait_limit_ns, abort_flag)) {
           if (!*abort_flag) ab.raise(p.status, kErrMmaWait);
           break;
@@ -212,8 +307,11 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tc_fence_after();
         const uint32_t d_i32 = tmem_base + buf * C::kAccCols;
         const uint32_t d_f32 = d_i32 + BN;
+        int kb0, kb_i8;
+        kb_range(tile, kb0, kb_i8);
+        const int kb_total = kb_i8 + kb_o;
         bool ok = true;
-        for (int kb = 0; kb < kb_total; ++kb) {
+        for (int kb = kb0; kb < kb_total; ++kb) {
           if (!wait_or_abort(full + stage, phase, p.wait_limit_ns, abort_flag)) {
             if (!*abort_flag) ab.raise(p.status, kErrMmaWait);
             ok = false;
@@ -226,7 +324,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
             for (int k = 0; k < kBK / 32; ++k)
               mma_i8(d_i32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescI8,
-                     (kb | k) != 0);
+                     (kb != kb0 || k != 0) ? 1u : 0u);
           } else {
             const int ko = kb - kb_i8;
 #pragma unroll
@@ -249,12 +347,31 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad+32)
+    // 8 warps: warp w reads TMEM lanes [32*(w%4), +32) (one output row per thread) and
+    // the column half (w-2)/4 of the tile, 32 columns at a time. The whole half-row is
+    // dequantized into registers (packed bf16) first, so the accumulator is handed back
+    // to the MMA warp before the stores; each 32x32 bf16 box then goes through this warp's
+    // staging buffer in shared memory to a TMA store.
+    constexpr int kChunks = BN / 64;  // 32-column chunks per warp
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
+    uint8_t* stage_tiles = epi_base + (warp - 2) * kEpiBufs * kStageTileBytes;
+    int ebuf = 0;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-      const int buf = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
+      const int buf = it % ACC_BUFS;
+      const uint32_t acc_phase = (it / ACC_BUFS) & 1;
+      // everything that does not need the accumulator is fetched before waiting for it
+      const int tile_mn = tile % mn_tiles;
+      const int split = tile / mn_tiles;
+      const int64_t m_tile0 = static_cast<int64_t>(tile_mn % p.num_m_tiles) * kBM;
+      const int64_t m = m_tile0 + row;
+      const int64_t n_half0 = static_cast<int64_t>(tile_mn / p.num_m_tiles) * BN + half * (BN / 2);
+      const bool m_ok = m < p.M;
+      const float d_m = m_ok ? __ldg(p.x_scale + m) : 0.0f;
+      const ColConsts cc = load_col_consts(p, n_half0, lane, kChunks);
+      const bool has_bias = p.bias != nullptr;
       // lane 0 waits and the warp follows its verdict, so the warp stays converged
       int ok = 0;
       if (lane == 0) {
@@ -264,80 +381,131 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const int64_t m = static_cast<int64_t>(tile % p.num_m_tiles) * kBM + row;
-      const int64_t n_tile0 = static_cast<int64_t>(tile / p.num_m_tiles) * BN;
-      const bool m_ok = m < p.M;
-      const float d_m = m_ok ? __ldg(p.x_scale + m) : 0.0f;
-      const float e_all = p.w_per_channel ? 0.0f : __ldg(p.w_scale);
-      const uint32_t t_i32 = tmem_base + buf * C::kAccCols + (static_cast<uint32_t>(quad * 32) << 16);
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        __syncwarp();
-        uint32_t acc[32];
-        uint32_t of[32];
-        tmem_ld_32x32b_x32(t_i32 + c * 32, acc);
-        if constexpr (OUTLIERS) {
-          if (kb_o > 0) tmem_ld_32x32b_x32(t_i32 + BN + c * 32, of);
-        }
-        tmem_wait_ld();
-        const int64_t n0 = n_tile0 + c * 32;
-        if (m_ok && n0 < p.N) {
-          const int nvalid = (p.N - n0) < 32 ? static_cast<int>(p.N - n0) : 32;  // a multiple of 8
-          float y[32];
+      const uint32_t t_row =
+          tmem_base + buf * C::kAccCols + (static_cast<uint32_t>(quad * 32) << 16) + half * (BN / 2);
+      if (p.splits == 1) {
+        uint32_t packed[kChunks][16];
 #pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            float4 e4 = make_float4(e_all, e_all, e_all, e_all);
-            if (p.w_per_channel && j < nvalid) e4 = __ldg(reinterpret_cast<const float4*>(p.w_scale + n0 + j));
-            const float e[4] = {e4.x, e4.y, e4.z, e4.w};
+        for (int c = 0; c < kChunks; ++c) {
+          const int64_t n0 = n_half0 + c * 32;
+          if (n0 < p.N) {  // uniform across the warp
+            __syncwarp();
+            uint32_t acc[32];
+            tmem_ld_32x32b_x32(t_row + c * 32, acc);
+            tmem_wait_ld();
+            const int nvalid = (p.N - n0) < 32 ? static_cast<int>(p.N - n0) : 32;  // a multiple of 8
+            float y[32];
+            dequant32(acc, d_m, cc, c, y);
+            if (p.acc_out != nullptr && m_ok) {
+              int32_t* arow = p.acc_out + m * p.N + n0;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              float v = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(acc[j + u])), d_m), e[u]);
-              if constexpr (OUTLIERS) {
-                if (kb_o > 0) v = __fadd_rn(v, __uint_as_float(of[j + u]));
+              for (int j = 0; j < 32; j += 4) {
+                if (j < nvalid)
+                  *reinterpret_cast<uint4*>(arow + j) = make_uint4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
               }
-              y[j + u] = v;
+            }
+            if constexpr (OUTLIERS) {
+              if (kb_o > 0) {
+                uint32_t of[32];  // fp32 outlier product of the same 32 columns
+                tmem_ld_32x32b_x32(t_row + BN + c * 32, of);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) y[j] = __fadd_rn(y[j], __uint_as_float(of[j]));
+              }
+            }
+            bias_pack32(y, has_bias, cc, c, packed[c]);
+          }
+        }
+        // the accumulator is no longer needed: hand it back before storing
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tmem_empty + buf);
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          const int64_t n0 = n_half0 + c * 32;
+          if (n0 < p.N) store_box(packed[c], stage_tiles, ebuf, lane, &tmY, n0, m_tile0 + quad * 32);
+        }
+      } else {
+        // K split: this split's int32 partial goes to the workspace; the warp that brings
+        // the last split of its 32-row x BN/2 sub-tile sums all partials (exact) and stores Y.
+        int32_t* part = p.partials + static_cast<int64_t>(split) * p.M * p.N;
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          const int64_t n0 = n_half0 + c * 32;
+          if (n0 < p.N) {
+            __syncwarp();
+            uint32_t acc[32];
+            tmem_ld_32x32b_x32(t_row + c * 32, acc);
+            tmem_wait_ld();
+            const int nvalid = (p.N - n0) < 32 ? static_cast<int>(p.N - n0) : 32;
+            if (m_ok) {
+              int32_t* prow = part + m * p.N + n0;
+#pragma unroll
+              for (int j = 0; j < 32; j += 4) {
+                if (j < nvalid)
+                  __stcg(reinterpret_cast<int4*>(prow + j), make_int4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]));
+              }
             }
           }
-          if (p.bias != nullptr) {
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tmem_empty + buf);
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+          int32_t* ctr = p.counters + static_cast<int64_t>(tile_mn) * kEpiWarps + (warp - 2);
+          if (atomicAdd(ctr, 1) == p.splits - 1) {
+            last = 1;
+            atomicExch(ctr, 0);  // leave the counter at zero for the next call
+          }
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          __threadfence();
+#pragma unroll 1
+          for (int c = 0; c < kChunks; ++c) {
+            const int64_t n0 = n_half0 + c * 32;
+            if (n0 >= p.N) break;
+            const int nvalid = (p.N - n0) < 32 ? static_cast<int>(p.N - n0) : 32;
+            uint32_t acc[32];
 #pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-              if (j < nvalid) {
-                const uint4 b = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + j));
-                const uint32_t w[4] = {b.x, b.y, b.z, b.w};
+            for (int j = 0; j < 32; ++j) acc[j] = 0;
+            if (m_ok) {
+              for (int sidx = 0; sidx < p.splits; ++sidx) {
+                const int32_t* prow = p.partials + (static_cast<int64_t>(sidx) * p.M + m) * p.N + n0;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  y[j + 2 * u] = __fadd_rn(y[j + 2 * u], __uint_as_float(w[u] << 16));
-                  y[j + 2 * u + 1] = __fadd_rn(y[j + 2 * u + 1], __uint_as_float(w[u] & 0xFFFF0000u));
+                for (int j = 0; j < 32; j += 4) {
+                  if (j < nvalid) {
+                    const int4 v = __ldcg(reinterpret_cast<const int4*>(prow + j));
+                    acc[j] += static_cast<uint32_t>(v.x);
+                    acc[j + 1] += static_cast<uint32_t>(v.y);
+                    acc[j + 2] += static_cast<uint32_t>(v.z);
+                    acc[j + 3] += static_cast<uint32_t>(v.w);
+                  }
                 }
               }
             }
-          }
-          uint16_t* yrow = p.Y + m * p.N + n0;
+            float y[32];
+            dequant32(acc, d_m, cc, c, y);
+            if (p.acc_out != nullptr && m_ok) {
+              int32_t* arow = p.acc_out + m * p.N + n0;
 #pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            if (j < nvalid) {
-              uint4 o;
-              o.x = pack_bf16x2(y[j + 0], y[j + 1]);
-              o.y = pack_bf16x2(y[j + 2], y[j + 3]);
-              o.z = pack_bf16x2(y[j + 4], y[j + 5]);
-              o.w = pack_bf16x2(y[j + 6], y[j + 7]);
-              *reinterpret_cast<uint4*>(yrow + j) = o;
+              for (int j = 0; j < 32; j += 4) {
+                if (j < nvalid)
+                  *reinterpret_cast<uint4*>(arow + j) = make_uint4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+              }
             }
-          }
-          if (p.acc_out != nullptr) {
-            int32_t* arow = p.acc_out + m * p.N + n0;
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              if (j < nvalid)
-                *reinterpret_cast<uint4*>(arow + j) = make_uint4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-            }
+            uint32_t packed[16];
+            bias_pack32(y, has_bias, cc, c, packed);
+            store_box(packed, stage_tiles, ebuf, lane, &tmY, n0, m_tile0 + quad * 32);
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tmem_empty + buf);
     }
+    // the output stores of this warp have completed before the CTA exits
+    if (lane == 0) bulk_wait_group<0>();
   }
 
   __syncwarp();
@@ -362,19 +530,25 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D K-major map: inner extent `inner` elements (contiguous), `outer` rows, row pitch
-// `pitch_bytes`; box = 128 bytes of K x box_rows rows, 128-byte swizzle, zero OOB fill.
-bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t inner,
-              uint64_t outer, uint64_t pitch_bytes, uint32_t box_rows) {
+// 2-D map: inner extent `inner` elements (contiguous), `outer` rows, row pitch `pitch_bytes`,
+// box = box_inner x box_rows elements; zero fill out of range.
+bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+              uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {pitch_bytes};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK / elem_bytes), box_rows};
+  const cuuint32_t box[2] = {box_inner, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// K-major operand map: 128 bytes of K x box_rows rows, 128-byte swizzle.
+bool make_operand_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t inner,
+                      uint64_t outer, uint64_t pitch_bytes, uint32_t box_rows) {
+  return make_map(map, base, dt, inner, outer, pitch_bytes, static_cast<uint32_t>(kBK / elem_bytes), box_rows,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 int num_sms() {
@@ -384,20 +558,56 @@ int num_sms() {
   return sms;
 }
 
-template <int BN, bool OUTLIERS>
-cudaError_t run(const GemmArgs& a, cudaStream_t stream, const char** why) {
-  using C = Cfg<BN, OUTLIERS>;
-  CUtensorMap tmA{}, tmB{}, tmXo{}, tmWo{};
+struct Plan {
+  int bn;
+  int splits;
+  int kb_per_split;
+};
+
+constexpr int kPlanSms = 148;  // planning is device-independent so workspace sizes are too
+
+Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool outliers) {
+  const int64_t m_t = (M + kBM - 1) / kBM;
+  const int64_t kb = (K + kBK - 1) / kBK;
+  auto tiles = [&](int bn) { return m_t * ((N + bn - 1) / bn); };
+  Plan pl{64, 1, static_cast<int>(kb)};
+  if (tiles(256) >= kPlanSms) {
+    pl.bn = 256;
+  } else if (tiles(128) >= kPlanSms) {
+    pl.bn = 128;
+  } else if (!outliers) {
+    const int64_t base = tiles(64);
+    if (2 * base <= kPlanSms && kb >= 4) {
+      int64_t sp = std::min<int64_t>({kPlanSms / base, kb / 2, 16});
+      const int64_t per = (kb + sp - 1) / sp;
+      pl.splits = static_cast<int>((kb + per - 1) / per);
+      pl.kb_per_split = static_cast<int>(per);
+    }
+  }
+  return pl;
+}
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+template <int BN, bool OUTLIERS, int ACC_BUFS>
+cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const char** why) {
+  using C = Cfg<BN, OUTLIERS, ACC_BUFS>;
+  CUtensorMap tmA{}, tmB{}, tmXo{}, tmWo{}, tmY{};
   const uint64_t K = static_cast<uint64_t>(a.K);
-  if (!make_map(&tmA, a.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, a.M, K, kBM) ||
-      !make_map(&tmB, a.Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, a.N, K, BN)) {
+  if (!make_operand_map(&tmA, a.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, a.M, K, kBM) ||
+      !make_operand_map(&tmB, a.Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, a.N, K, BN)) {
     *why = "cuTensorMapEncodeTiled failed for the int8 operands";
+    return cudaErrorInvalidValue;
+  }
+  if (!make_map(&tmY, a.Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.M),
+                static_cast<uint64_t>(a.N) * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+    *why = "cuTensorMapEncodeTiled failed for the output";
     return cudaErrorInvalidValue;
   }
   if (OUTLIERS) {
     const uint64_t ldo = static_cast<uint64_t>(a.ld_o);
-    if (!make_map(&tmXo, a.Xo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ldo, a.M, ldo * 2, kBM) ||
-        !make_map(&tmWo, a.Wo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ldo, a.N, ldo * 2, BN)) {
+    if (!make_operand_map(&tmXo, a.Xo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ldo, a.M, ldo * 2, kBM) ||
+        !make_operand_map(&tmWo, a.Wo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ldo, a.N, ldo * 2, BN)) {
       *why = "cuTensorMapEncodeTiled failed for the outlier operands";
       return cudaErrorInvalidValue;
     }
@@ -410,7 +620,7 @@ cudaError_t run(const GemmArgs& a, cudaStream_t stream, const char** why) {
   cudaGetDevice(&dev);
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_done.load() & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(w8a8_gemm_kernel<BN, OUTLIERS>,
+    cudaError_t e = cudaFuncSetAttribute(w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) {
       *why = "cudaFuncSetAttribute(MaxDynamicSharedMemorySize) failed";
@@ -423,39 +633,53 @@ cudaError_t run(const GemmArgs& a, cudaStream_t stream, const char** why) {
   p.w_scale = a.w_scale;
   p.w_per_channel = a.w_per_channel ? 1 : 0;
   p.bias = a.bias;
-  p.Y = a.Y;
   p.acc_out = a.acc_out;
   p.M = a.M;
   p.N = a.N;
   p.num_m_tiles = static_cast<int>((a.M + kBM - 1) / kBM);
   p.num_n_tiles = static_cast<int>((a.N + BN - 1) / BN);
   p.num_kb = static_cast<int>((a.K + kBK - 1) / kBK);
+  p.splits = pl.splits;
+  p.kb_per_split = pl.kb_per_split;
+  p.partials = nullptr;
+  p.counters = nullptr;
+  if (pl.splits > 1) {
+    p.partials = static_cast<int32_t*>(a.ws);
+    p.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(a.ws) +
+                                            up256(sizeof(int32_t) * pl.splits * a.M * a.N));
+  }
   p.o_count = a.o_count;
   p.status = device_status_word();
   p.wait_limit_ns = a.wait_limit_ns;
   p.fault = a.fault;
-  const int tiles = p.num_m_tiles * p.num_n_tiles;
+  const int tiles = p.num_m_tiles * p.num_n_tiles * p.splits;
   const int grid = std::min(tiles, num_sms());
   note_launch();
-  w8a8_gemm_kernel<BN, OUTLIERS><<<grid, kThreads, C::kSmemBytes, stream>>>(tmA, tmB, tmXo, tmWo, p);
+  w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS><<<grid, kThreads, C::kSmemBytes, stream>>>(tmA, tmB, tmXo, tmWo, tmY, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t gemm_workspace_bytes(int64_t, int64_t, int64_t, bool) { return 0; }
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, bool outliers) {
+  const Plan pl = plan_gemm(M, N, K, outliers);
+  if (pl.splits == 1) return 0;
+  const int64_t tiles_mn = ((M + kBM - 1) / kBM) * ((N + pl.bn - 1) / pl.bn);
+  return up256(sizeof(int32_t) * pl.splits * M * N) + up256(sizeof(int32_t) * tiles_mn * kEpiWarps);
+}
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream, const char** why) {
-  const int sms = num_sms();
-  const int64_t m_tiles = (a.M + kBM - 1) / kBM;
-  auto tiles = [&](int bn) { return m_tiles * ((a.N + bn - 1) / bn); };
-  if (a.Xo != nullptr) {
-    if (tiles(128) >= sms) return run<128, true>(a, stream, why);
-    return run<64, true>(a, stream, why);
+  const bool outliers = a.Xo != nullptr;
+  const Plan pl = plan_gemm(a.M, a.N, a.K, outliers);
+  if (outliers) {
+    // int32 + fp32 accumulators: 256-wide tiles fit TMEM once, narrower ones twice
+    if (pl.bn == 256) return run<256, true, 1>(a, pl, stream, why);
+    if (pl.bn == 128) return run<128, true, 2>(a, pl, stream, why);
+    return run<64, true, 2>(a, pl, stream, why);
   }
-  if (tiles(256) >= sms) return run<256, false>(a, stream, why);
-  if (tiles(128) >= sms) return run<128, false>(a, stream, why);
-  return run<64, false>(a, stream, why);
+  if (pl.bn == 256) return run<256, false, 2>(a, pl, stream, why);
+  if (pl.bn == 128) return run<128, false, 2>(a, pl, stream, why);
+  return run<64, false, 2>(a, pl, stream, why);
 }
 
 }  // namespace sq

@@ -24,30 +24,6 @@ namespace {
 
 constexpr int kCta = 256;
 
-__device__ __forceinline__ void load16(const uint16_t* p, float (&v)[16]) {
-  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
-  const uint4 b = __ldg(reinterpret_cast<const uint4*>(p + 8));
-  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    v[2 * i] = __uint_as_float(w[i] << 16);
-    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-
-__device__ __forceinline__ void scale16(const float* __restrict__ vec, int64_t k, float (&v)[16]) {
-  if (vec == nullptr) return;
-  const float4* p = reinterpret_cast<const float4*>(vec + k);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float4 f = __ldg(p + i);
-    v[4 * i + 0] = __fmul_rn(v[4 * i + 0], f.x);
-    v[4 * i + 1] = __fmul_rn(v[4 * i + 1], f.y);
-    v[4 * i + 2] = __fmul_rn(v[4 * i + 2], f.z);
-    v[4 * i + 3] = __fmul_rn(v[4 * i + 3], f.w);
-  }
-}
-
 // 16 skip bits for columns k..k+15 (k % 16 == 0).
 __device__ __forceinline__ uint32_t skip_bits16(const uint32_t* __restrict__ mask, int64_t k) {
   return (__ldg(mask + (k >> 5)) >> (k & 31)) & 0xFFFFu;
@@ -95,106 +71,213 @@ __device__ __forceinline__ float group_max(float a, float* red /* [kCta/32] */) 
 
 enum Mode { kPerRow = 0, kTensorMax = 1, kTensorQuant = 2 };
 
-// Load 16 elements of a row starting at column k, zero the LLM.int8 outlier columns
-// (copying their bf16 values to the gathered matrix when `gather`), then smooth.
-template <bool OUTLIERS>
-__device__ __forceinline__ void load_chunk(const uint16_t* __restrict__ srow, int64_t row, int64_t k,
-                                           const float* __restrict__ vec, const OutlierView& ov, bool gather,
-                                           float (&v)[16]) {
-  load16(srow + k, v);
+__device__ __forceinline__ void raw16(const uint16_t* p, uint4 (&r)[2]) {
+  r[0] = __ldg(reinterpret_cast<const uint4*>(p));
+  r[1] = __ldg(reinterpret_cast<const uint4*>(p + 8));
+}
+
+__device__ __forceinline__ void widen16(const uint4 (&r)[2], float (&v)[16]) {
+  const uint32_t w[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// Zero the LLM.int8 outlier columns among k..k+15 (copying their bf16 values to the gathered
+// matrix when `gather`), then smooth with the thread's slice of the vector (if any).
+template <bool OUTLIERS, bool HAS_VEC>
+__device__ __forceinline__ void finish_chunk(const uint4 (&r)[2], int64_t row, int64_t k, const float (&vs)[16],
+                                             const OutlierView& ov, bool gather, float (&v)[16]) {
+  widen16(r, v);
   if constexpr (OUTLIERS) {
     const uint32_t sk = skip_bits16(ov.mask, k);
     if (sk) {
       const int64_t w = k >> 5;
       int32_t pos = __ldg(ov.prefix + w) + __popc(__ldg(ov.mask + w) & ((1u << (k & 31)) - 1u));
+      const uint16_t* h = reinterpret_cast<const uint16_t*>(&r[0]);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         if ((sk >> i) & 1u) {
-          if (gather) ov.gathered[row * ov.ld_gathered + pos] = srow[k + i];
+          if (gather) ov.gathered[row * ov.ld_gathered + pos] = h[i];
           ++pos;
           v[i] = 0.0f;
         }
       }
     }
   }
-  scale16(vec, k, v);
+  if constexpr (HAS_VEC) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], vs[i]);
+  }
 }
 
-// Grid: one row group per (blockIdx.x, threadIdx.x / TPR); CTA = max(kCta, TPR) threads.
-template <int TPR, int CHUNKS, bool TWO_PASS, bool OUTLIERS, int MODE>
+// Persistent over rows: CTA = max(kCta, TPR) threads = kGroups row groups of TPR threads;
+// the groups walk the rows with a grid stride. A thread keeps its slice of the smoothing
+// vector in registers for all its rows and prefetches its next row's bf16 data before the
+// current row's absmax reduction.
+template <int TPR, int CHUNKS, bool TWO_PASS, bool OUTLIERS, bool HAS_VEC, int MODE>
 __global__ void __launch_bounds__(TPR > kCta ? TPR : kCta)
 quant_rows_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
                   const float* __restrict__ vec, OutlierView ov, int8_t* __restrict__ q,
                   float* __restrict__ scale, unsigned int* __restrict__ gmax_bits) {
   constexpr int kThreads = TPR > kCta ? TPR : kCta;
   constexpr int kGroups = kThreads / TPR;
+  constexpr int kVC = (HAS_VEC && !TWO_PASS) ? CHUNKS : 1;
   __shared__ float red[kThreads / 32];
   const int g = threadIdx.x / TPR;
   const int t = threadIdx.x % TPR;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * kGroups + g;
-  const bool row_ok = row < rows;
-  const uint16_t* srow = src + (row_ok ? row : 0) * ld;
   const int64_t step = static_cast<int64_t>(TPR) * 16;
+  const int64_t row_stride = static_cast<int64_t>(gridDim.x) * kGroups;
 
-  float a = 0.0f;
-  float v[TWO_PASS ? 1 : CHUNKS][16];
-  if constexpr (!TWO_PASS) {
+  float vs[kVC][16];
+  if constexpr (HAS_VEC && !TWO_PASS) {
 #pragma unroll
     for (int c = 0; c < CHUNKS; ++c) {
       const int64_t k = c * step + t * 16;
-      if (row_ok && k < K) {
-        load_chunk<OUTLIERS>(srow, row, k, vec, ov, MODE != kTensorMax, v[c]);
+      if (k < K) {
+        const float4* p4 = reinterpret_cast<const float4*>(vec + k);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[c][i]));
+        for (int i = 0; i < 4; ++i) {
+          const float4 f = __ldg(p4 + i);
+          vs[c][4 * i] = f.x;
+          vs[c][4 * i + 1] = f.y;
+          vs[c][4 * i + 2] = f.z;
+          vs[c][4 * i + 3] = f.w;
+        }
       }
-    }
-  } else if constexpr (MODE != kTensorQuant) {
-    for (int64_t k = t * 16; row_ok && k < K; k += step) {
-      float w[16];
-      load_chunk<OUTLIERS>(srow, row, k, vec, ov, false, w);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(w[i]));
     }
   }
 
-  if constexpr (MODE == kTensorQuant) {
-    a = __uint_as_float(*reinterpret_cast<volatile unsigned int*>(gmax_bits));
-  } else {
-    a = group_max<TPR>(a, red);
+  uint4 raw[TWO_PASS ? 1 : CHUNKS][2];
+  int64_t row = static_cast<int64_t>(blockIdx.x) * kGroups + g;
+  if constexpr (!TWO_PASS) {
+    if (row < rows) {
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) {
+        const int64_t k = c * step + t * 16;
+        if (k < K) raw16(src + row * ld + k, raw[c]);
+      }
+    }
   }
 
-  if constexpr (MODE == kTensorMax) {
-    if (t == 0 && row_ok) atomicMax(gmax_bits, __float_as_uint(a));
-  } else {
-    const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
-    if (row_ok) {
-      if constexpr (MODE == kPerRow) {
-        if (t == 0) scale[row] = __fdiv_rn(a, 127.0f);
-      } else {
-        if (t == 0 && row == 0) scale[0] = __fdiv_rn(a, 127.0f);
+  // uniform trip count across the CTA (block-wide reductions inside)
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kGroups; base < rows; base += row_stride, row += row_stride) {
+    const bool row_ok = row < rows;
+    const uint16_t* srow = src + (row_ok ? row : 0) * ld;
+    float a = 0.0f;
+    float v[TWO_PASS ? 1 : CHUNKS][16];
+    if constexpr (!TWO_PASS) {
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) {
+        const int64_t k = c * step + t * 16;
+        if (row_ok && k < K) {
+          finish_chunk<OUTLIERS, HAS_VEC>(raw[c], row, k, vs[HAS_VEC ? c : 0], ov, MODE != kTensorMax, v[c]);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[c][i]));
+        }
       }
-      int8_t* qrow = q + row * K;
-      if constexpr (!TWO_PASS) {
+      // prefetch this thread's next row while the current one is reduced
+      const int64_t nrow = row + row_stride;
+      if (nrow < rows) {
 #pragma unroll
         for (int c = 0; c < CHUNKS; ++c) {
           const int64_t k = c * step + t * 16;
-          if (k < K) store_q16(qrow + k, v[c], r);
-        }
-      } else {
-        for (int64_t k = t * 16; k < K; k += step) {
-          float w[16];
-          load_chunk<OUTLIERS>(srow, row, k, vec, ov, true, w);
-          store_q16(qrow + k, w, r);
+          if (k < K) raw16(src + nrow * ld + k, raw[c]);
         }
       }
-      if constexpr (OUTLIERS) {
-        // zero the padding of the gathered row up to the next multiple of 64 columns
-        const int32_t cnt = __ldg(ov.count);
-        const int32_t padded = (cnt + 63) & ~63;
-        for (int32_t c = cnt + t; c < padded; c += TPR) ov.gathered[row * ov.ld_gathered + c] = 0;
+    } else if constexpr (MODE != kTensorQuant) {
+      for (int64_t k = t * 16; row_ok && k < K; k += step) {
+        uint4 r[2];
+        float w[16], vv[16];
+        raw16(srow + k, r);
+        if constexpr (HAS_VEC) {
+          const float4* p4 = reinterpret_cast<const float4*>(vec + k);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 f = __ldg(p4 + i);
+            vv[4 * i] = f.x; vv[4 * i + 1] = f.y; vv[4 * i + 2] = f.z; vv[4 * i + 3] = f.w;
+          }
+        }
+        finish_chunk<OUTLIERS, HAS_VEC>(r, row, k, vv, ov, false, w);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(w[i]));
+      }
+    }
+
+    if constexpr (MODE == kTensorQuant) {
+      a = __uint_as_float(*reinterpret_cast<volatile unsigned int*>(gmax_bits));
+    } else {
+      a = group_max<TPR>(a, red);
+    }
+
+    if constexpr (MODE == kTensorMax) {
+      if (t == 0 && row_ok) atomicMax(gmax_bits, __float_as_uint(a));
+    } else {
+      const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+      if (row_ok) {
+        if constexpr (MODE == kPerRow) {
+          if (t == 0) scale[row] = __fdiv_rn(a, 127.0f);
+        } else {
+          if (t == 0 && row == 0) scale[0] = __fdiv_rn(a, 127.0f);
+        }
+        int8_t* qrow = q + row * K;
+        if constexpr (!TWO_PASS) {
+#pragma unroll
+          for (int c = 0; c < CHUNKS; ++c) {
+            const int64_t k = c * step + t * 16;
+            if (k < K) store_q16(qrow + k, v[c], r);
+          }
+        } else {
+          for (int64_t k = t * 16; k < K; k += step) {
+            uint4 rr[2];
+            float w[16], vv[16];
+            raw16(srow + k, rr);
+            if constexpr (HAS_VEC) {
+              const float4* p4 = reinterpret_cast<const float4*>(vec + k);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float4 f = __ldg(p4 + i);
+                vv[4 * i] = f.x; vv[4 * i + 1] = f.y; vv[4 * i + 2] = f.z; vv[4 * i + 3] = f.w;
+              }
+            }
+            finish_chunk<OUTLIERS, HAS_VEC>(rr, row, k, vv, ov, true, w);
+            store_q16(qrow + k, w, r);
+          }
+        }
+        if constexpr (OUTLIERS) {
+          // zero the padding of the gathered row up to the next multiple of 64 columns
+          const int32_t cnt = __ldg(ov.count);
+          const int32_t padded = (cnt + 63) & ~63;
+          for (int32_t c = cnt + t; c < padded; c += TPR) ov.gathered[row * ov.ld_gathered + c] = 0;
+        }
       }
     }
   }
+}
+
+int num_sms() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  return sms;
+}
+
+// One resident wave: as many CTAs as fit on every SM at once (registers decide); the
+// row-group loop and the prefetch of the next row keep the loads in flight.
+template <typename Kernel>
+int64_t resident_grid(Kernel kernel, int threads, int64_t groups, int& per_sm_cache) {
+  if (per_sm_cache <= 0) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1)
+      per_sm = 1;
+    per_sm_cache = per_sm;
+  }
+  return std::min<int64_t>(groups, static_cast<int64_t>(num_sms()) * per_sm_cache);
 }
 
 template <int TPR, int CHUNKS, bool TWO_PASS, bool OUTLIERS, int MODE>
@@ -202,15 +285,24 @@ cudaError_t launch_t(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, c
                      const OutlierView& ov, int8_t* q, float* scale, unsigned int* gmax, cudaStream_t stream) {
   constexpr int kThreads = TPR > kCta ? TPR : kCta;
   constexpr int kGroups = kThreads / TPR;
-  const int64_t blocks = (rows + kGroups - 1) / kGroups;
+  const int64_t groups = (rows + kGroups - 1) / kGroups;
   note_launch();
-  quant_rows_kernel<TPR, CHUNKS, TWO_PASS, OUTLIERS, MODE>
-      <<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(src, rows, K, ld, vec, ov, q, scale, gmax);
+  if (vec != nullptr) {
+    static int per_sm = 0;
+    auto kernel = quant_rows_kernel<TPR, CHUNKS, TWO_PASS, OUTLIERS, true, MODE>;
+    const int64_t blocks = resident_grid(kernel, kThreads, groups, per_sm);
+    kernel<<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(src, rows, K, ld, vec, ov, q, scale, gmax);
+  } else {
+    static int per_sm = 0;
+    auto kernel = quant_rows_kernel<TPR, CHUNKS, TWO_PASS, OUTLIERS, false, MODE>;
+    const int64_t blocks = resident_grid(kernel, kThreads, groups, per_sm);
+    kernel<<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(src, rows, K, ld, vec, ov, q, scale, gmax);
+  }
   return cudaGetLastError();
 }
 
-// Shape dispatch: the smallest threads-per-row that keeps <= 32 (<= 64 for long rows)
-// smoothed values per thread in registers.
+// Shape dispatch: the smallest threads-per-row that keeps <= 32 smoothed values per thread
+// in registers; rows longer than 16384 take the two-read path.
 template <bool OUTLIERS, int MODE>
 cudaError_t dispatch(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, const float* vec,
                      const OutlierView& ov, int8_t* q, float* scale, unsigned int* gmax, cudaStream_t stream) {

@@ -106,11 +106,11 @@ cudaError_t launch_col_absmax(const uint16_t* src, int64_t rows, int64_t K, int6
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t col_blocks = (K + kColsPerCta - 1) / kColsPerCta;
-  // about 8 resident CTAs per SM and 2 waves; at least 8 rows (one per warp) per CTA
-  const int64_t target = static_cast<int64_t>(sms) * 16;
+  // one wave of ~4 CTAs per SM, at least 64 rows per CTA (few atomics per column)
+  const int64_t target = static_cast<int64_t>(sms) * 4;
   int64_t row_blocks = std::max<int64_t>(1, target / col_blocks);
   int64_t rows_per_cta = (rows + row_blocks - 1) / row_blocks;
-  rows_per_cta = std::max<int64_t>(kColWarps, ((rows_per_cta + kColWarps - 1) / kColWarps) * kColWarps);
+  rows_per_cta = std::max<int64_t>(64, ((rows_per_cta + kColWarps - 1) / kColWarps) * kColWarps);
   row_blocks = (rows + rows_per_cta - 1) / rows_per_cta;
   if (row_blocks > 65535) {
     row_blocks = 65535;

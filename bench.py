@@ -40,8 +40,8 @@ N_SETS = 4  # rotating input sets: 4 x (16.8 MB X + 90.2 MB W) = 428 MB > 126 MB
 
 # DRAM traffic of one int8 GEMM launch on this workload, from the committed ncu capture
 # (profiles/int8_gemm_llama7b_mlp_up.md), valid while the GEMM source hashes to GEMM_SRC_SHA.
-NCU_GEMM_TRAFFIC_BYTES = None
-GEMM_SRC_SHA = None
+NCU_GEMM_TRAFFIC_BYTES = 53605888 + 11876608
+GEMM_SRC_SHA = "63a2219cee91fc70"
 
 
 def _peaks():
@@ -254,8 +254,10 @@ def run_ours(args):
 
     # ---------------------------------------------------------------- timed region
     # The K timed steps are captured once as one CUDA graph (launch overhead out of the way,
-    # as a serving loop would run them), with timing events between the operations of every
-    # step; the graph is replayed once untimed and once timed.
+    # as a serving loop would run them); every SAMPLE_EVERY-th step carries timing events
+    # between its operations (an event node costs a few microseconds inside a graph, so
+    # instrumenting every step would inflate the step time). The graph is replayed once
+    # untimed and once timed.
     records = []
     mode = "cuda_graph"
     stream = torch.cuda.Stream()
@@ -265,7 +267,7 @@ def run_ours(args):
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=stream):
             for i in range(args.steps):
-                path.step(i, records, external=True)
+                path.step(i, records if i % args.sample_every == 0 else None, external=True)
         launches = sq.sq_kernel_launch_count() - launches0
         with torch.cuda.stream(stream):
             graph.replay()
@@ -289,7 +291,7 @@ def run_ours(args):
                 launches0 = sq.sq_kernel_launch_count()
                 t_start.record()
                 for i in range(args.steps):
-                    path.step(i, records)
+                    path.step(i, records if i % args.sample_every == 0 else None)
                 t_end.record()
                 launches = sq.sq_kernel_launch_count() - launches0
         torch.cuda.synchronize()
@@ -346,6 +348,8 @@ def run_ours(args):
                    "l2": f"{N_SETS} rotating input sets ({N_SETS * (2 * M * K + 2 * N * K) / 1e6:.0f} MB) > L2",
                    "parallelism": f"replica x{ws}"},
         "roofline": roofline, "kernels": kernels, "gpu_launches": int(launches), "launch_mode": mode,
+        "kernel_timing": f"CUDA event nodes around each operation of every {args.sample_every}th timed step "
+                         f"({len(records)} steps sampled)",
         "clocks": clk.summary(), "e2e": e2e, "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16, "kind": peak_kind},
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -485,6 +489,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--sample-every", type=int, default=10, help="timed steps per step carrying event nodes")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=64, help="token rows per reference-arm step")

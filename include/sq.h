@@ -135,12 +135,13 @@ SQ_API sq_status sq_quant_act_per_token(const void* X_bf16, int64_t M, int64_t K
  * Xq: int8 [M, K]; Wq: int8 [N, K]; x_scale: fp32 [M]; w_scale: fp32 [N] (SQ_PER_CHANNEL)
  * or [1] (SQ_PER_TENSOR); bias: bf16 [N] or NULL; Y: bf16 [M, N].
  * acc_out: int32 [M, N] or NULL — when given, the raw INT32 accumulator is written too
- * (for exact checking). ws: sq_workspace_size(SQ_OP_INT8_GEMM_DEQUANT, M, N, K) bytes, zero
+ * (for exact checking). ws: sq_workspace_size(SQ_OP_INT8_GEMM_DEQUANT, M, N, K) bytes: zero
  * for shapes with enough output tiles to fill the GPU (ws may then be NULL). Small-M shapes
- * split K across CTAs: each split writes exact int32 partials to ws and the last split to
- * arrive sums them and runs the epilogue. Such a ws must be zero-filled before its first use;
- * every completed call leaves its arrival counters at zero again (after SQ_ERR_TIMEOUT, zero
- * it again). Calls that share one ws must not overlap on the GPU.
+ * split every tile along K: each part writes its exact int32 partial to ws and the last part
+ * to arrive sums them and runs the epilogue, so the result is bit-identical to the unsplit
+ * one. Such a ws must be zero-filled before its first use; every completed call leaves its
+ * arrival counters at zero again (after SQ_ERR_TIMEOUT, zero it again). Calls that share
+ * one ws must not overlap on the GPU.
  */
 SQ_API sq_status sq_int8_gemm_dequant(const int8_t* Xq, const int8_t* Wq, const float* x_scale, const float* w_scale,
                                sq_gran w_gran, const void* bias_bf16, void* Y_bf16, int64_t M, int64_t N,

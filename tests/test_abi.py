@@ -44,7 +44,7 @@ def test_workspace_sizes():
     # int8 activations + gathered bf16 outlier operands (worst case: every column)
     assert ws >= M * K + 2 * (M + N) * K
     assert sq.sq_workspace_size(99, M, N, K) == 0
-    # enough output tiles: no split, no workspace; decode-sized M splits K over int32 partials
+    # enough output tiles to fill the GPU: whole tiles, no workspace
     assert sq.sq_workspace_size(sq.SQ_OP_INT8_GEMM_DEQUANT, M, N, K) == 0
     dec = sq.sq_workspace_size(sq.SQ_OP_INT8_GEMM_DEQUANT, 64, 4096, 4096)
     assert dec >= 2 * 64 * 4096 * 4

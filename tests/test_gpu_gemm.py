@@ -30,7 +30,8 @@ def _gemm_direct(xq, wq, d, e, gran, bias_bits):
 # BN = 64 / 128 / 256 variants (the variant depends on the tile count versus the SM count)
 # (128,128,4096), (257,1000,528), (3,200,1040) and (64,4096,4096) split K over int32 partials
 GEMM_SHAPES = [(1, 8, 16), (16, 256, 256), (5, 24, 48), (130, 72, 144), (200, 264, 208), (128, 128, 4096),
-               (257, 1000, 528), (3, 200, 1040), (64, 4096, 4096), (1024, 2048, 1024), (2304, 2120, 720)]
+               (257, 1000, 528), (3, 200, 1040), (64, 4096, 4096), (1024, 2048, 1024), (300, 9480, 528),
+               (2304, 2120, 720)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
@@ -78,6 +79,7 @@ def test_tiny_config_full_path(gran):
 
 
 @pytest.mark.parametrize("M,N,K,gran", [(77, 136, 528, sq.SQ_PER_CHANNEL), (300, 520, 1040, sq.SQ_PER_TENSOR),
+                                        (300, 9480, 528, sq.SQ_PER_TENSOR),
                                         (1, 4096, 4096, sq.SQ_PER_CHANNEL), (64, 1024, 4096, sq.SQ_PER_CHANNEL)])
 def test_smoothquant_path_ragged(M, N, K, gran):
     p = wl.random_problem(M, N, K, seed=M + N + K, outliers=3, offset=40.0, w_gran=gran)

@@ -30,7 +30,8 @@ def test_tiny_config_outliers_are_channels_0_1():
 
 
 @pytest.mark.parametrize("M,N,K,nout", [(5, 24, 48, 1), (130, 72, 144, 3), (200, 264, 208, 7),
-                                        (257, 1000, 528, 70), (1024, 2048, 1024, 10), (64, 4096, 4096, 6)])
+                                        (257, 1000, 528, 70), (1024, 2048, 1024, 10), (64, 4096, 4096, 6),
+                                        (300, 9480, 528, 5)])
 def test_random_ragged(M, N, K, nout):
     p = wl.random_problem(M, N, K, seed=M + 3 * N + K, outliers=nout, offset=25.0)
     g, _ = _check(p)

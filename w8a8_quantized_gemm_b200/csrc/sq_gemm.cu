@@ -64,10 +64,15 @@ struct Params {
   int32_t* acc_out;
   int64_t M, N;
   int num_m_tiles, num_n_tiles, num_kb;
-  int splits;          // K splits per output tile (1: no split)
-  int kb_per_split;    // k-blocks per split
-  int32_t* partials;   // [splits][M][N] int32 (splits > 1)
-  int32_t* counters;   // [m_tiles * n_tiles * kEpiWarps] arrival counters (splits > 1), zero between calls
+  // Work units: units [0, num_full) are whole output tiles (tile index = unit); the tiles
+  // after them ("tail" tiles) are split along K into `splits` units of kb_per_split k-blocks,
+  // whose exact int32 partials meet in the workspace.
+  int num_full;
+  int num_units;
+  int splits;
+  int kb_per_split;
+  int32_t* partials;   // [tail tiles * splits][kEpiWarps][BN/64 chunks][8][32 lanes] int4 (int32 x4)
+  int32_t* counters;   // [tail tiles * kEpiWarps] arrival counters, zero between calls
   const int32_t* o_count;
   unsigned int* status;
   uint64_t wait_limit_ns;
@@ -81,6 +86,32 @@ struct Abort {
     *flag = 1;
   }
 };
+
+struct Unit {
+  int tile_mn;  // output tile (m fastest)
+  int split;    // part of a split tail tile (0 for whole tiles)
+  int kb0, kb1; // int8 k-block range
+  bool is_split;
+};
+
+__device__ __forceinline__ Unit unit_of(const Params& p, int u) {
+  Unit w;
+  if (u < p.num_full) {
+    w.tile_mn = u;
+    w.split = 0;
+    w.kb0 = 0;
+    w.kb1 = p.num_kb;
+    w.is_split = false;
+  } else {
+    const int v = u - p.num_full;
+    w.tile_mn = p.num_full + v / p.splits;
+    w.split = v % p.splits;
+    w.kb0 = w.split * p.kb_per_split;
+    w.kb1 = min(p.num_kb, w.kb0 + p.kb_per_split);
+    w.is_split = true;
+  }
+  return w;
+}
 
 // Bounded wait that also gives up as soon as another role has aborted.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
@@ -228,16 +259,9 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  // tiles: m fastest, then n, then the K split
-  const int mn_tiles = p.num_m_tiles * p.num_n_tiles;
-  const int num_tiles = mn_tiles * p.splits;
+  const int num_units = p.num_units;
   int kb_o = 0;
   if constexpr (OUTLIERS) kb_o = (__ldg(p.o_count) + 63) / 64;
-  auto kb_range = [&](int tile, int& kb_begin, int& kb_i8_end) {
-    const int split = tile / mn_tiles;
-    kb_begin = split * p.kb_per_split;
-    kb_i8_end = min(p.num_kb, kb_begin + p.kb_per_split);
-  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -247,11 +271,11 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       uint32_t issued_mask = 0;      // stages that received at least one load
       uint32_t issued_parity = 0;    // parity of the last load issued into each stage
       bool withheld = false;
-      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
-        const int m0 = (tile % p.num_m_tiles) * kBM;
-        const int n0 = ((tile % mn_tiles) / p.num_m_tiles) * BN;
-        int kb0, kb_i8;
-        kb_range(tile, kb0, kb_i8);
+      for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
+        const Unit w = unit_of(p, u);
+        const int m0 = (w.tile_mn % p.num_m_tiles) * kBM;
+        const int n0 = (w.tile_mn / p.num_m_tiles) * BN;
+        const int kb0 = w.kb0, kb_i8 = w.kb1;
         const int kb_total = kb_i8 + kb_o;
         for (int kb = kb0; kb < kb_total; ++kb) {
           if (!wait_or_abort(empty + stage, phase ^ 1, p.wait_limit_ns, abort_flag)) {
@@ -297,7 +321,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, ++it) {
+      for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x, ++it) {
         const int buf = it % ACC_BUFS;
         const uint32_t acc_phase = (it / ACC_BUFS) & 1;
         if (!wait_or_abort(tmem_empty + buf, acc_phase ^ 1, p.wait_limit_ns, abort_flag)) {
@@ -307,8 +331,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tc_fence_after();
         const uint32_t d_i32 = tmem_base + buf * C::kAccCols;
         const uint32_t d_f32 = d_i32 + BN;
-        int kb0, kb_i8;
-        kb_range(tile, kb0, kb_i8);
+        const Unit w = unit_of(p, u);
+        const int kb0 = w.kb0, kb_i8 = w.kb1;
         const int kb_total = kb_i8 + kb_o;
         bool ok = true;
         for (int kb = kb0; kb < kb_total; ++kb) {
@@ -359,12 +383,13 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     uint8_t* stage_tiles = epi_base + (warp - 2) * kEpiBufs * kStageTileBytes;
     int ebuf = 0;
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+    for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++it) {
       const int buf = it % ACC_BUFS;
       const uint32_t acc_phase = (it / ACC_BUFS) & 1;
       // everything that does not need the accumulator is fetched before waiting for it
-      const int tile_mn = tile % mn_tiles;
-      const int split = tile / mn_tiles;
+      const Unit w = unit_of(p, u);
+      const int tile_mn = w.tile_mn;
+      const int split = w.split;
       const int64_t m_tile0 = static_cast<int64_t>(tile_mn % p.num_m_tiles) * kBM;
       const int64_t m = m_tile0 + row;
       const int64_t n_half0 = static_cast<int64_t>(tile_mn / p.num_m_tiles) * BN + half * (BN / 2);
@@ -383,7 +408,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       tc_fence_after();
       const uint32_t t_row =
           tmem_base + buf * C::kAccCols + (static_cast<uint32_t>(quad * 32) << 16) + half * (BN / 2);
-      if (p.splits == 1) {
+      if (!w.is_split) {
         uint32_t packed[kChunks][16];
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
@@ -428,7 +453,13 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       } else {
         // K split: this split's int32 partial goes to the workspace; the warp that brings
         // the last split of its 32-row x BN/2 sub-tile sums all partials (exact) and stores Y.
-        int32_t* part = p.partials + static_cast<int64_t>(split) * p.M * p.N;
+        // Partials are stored warp-contiguous (lane-minor), so every access moves 512 bytes.
+        const int64_t tail = tile_mn - p.num_full;
+        constexpr int64_t kSlotInt4 = static_cast<int64_t>(kEpiWarps) * kChunks * 8 * 32;
+        auto part_ptr = [&](int sidx, int c) {
+          return reinterpret_cast<int4*>(p.partials) + (tail * p.splits + sidx) * kSlotInt4 +
+                 ((static_cast<int64_t>(warp - 2) * kChunks + c) * 8) * 32 + lane;
+        };
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
           const int64_t n0 = n_half0 + c * 32;
@@ -437,15 +468,10 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             uint32_t acc[32];
             tmem_ld_32x32b_x32(t_row + c * 32, acc);
             tmem_wait_ld();
-            const int nvalid = (p.N - n0) < 32 ? static_cast<int>(p.N - n0) : 32;
-            if (m_ok) {
-              int32_t* prow = part + m * p.N + n0;
+            int4* dst = part_ptr(split, c);
 #pragma unroll
-              for (int j = 0; j < 32; j += 4) {
-                if (j < nvalid)
-                  __stcg(reinterpret_cast<int4*>(prow + j), make_int4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]));
-              }
-            }
+            for (int j = 0; j < 8; ++j)
+              __stcg(dst + j * 32, make_int4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]));
           }
         }
         tc_fence_before();
@@ -455,7 +481,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         __syncwarp();
         int last = 0;
         if (lane == 0) {
-          int32_t* ctr = p.counters + static_cast<int64_t>(tile_mn) * kEpiWarps + (warp - 2);
+          int32_t* ctr = p.counters + tail * kEpiWarps + (warp - 2);
           if (atomicAdd(ctr, 1) == p.splits - 1) {
             last = 1;
             atomicExch(ctr, 0);  // leave the counter at zero for the next call
@@ -472,19 +498,15 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             uint32_t acc[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) acc[j] = 0;
-            if (m_ok) {
-              for (int sidx = 0; sidx < p.splits; ++sidx) {
-                const int32_t* prow = p.partials + (static_cast<int64_t>(sidx) * p.M + m) * p.N + n0;
+            for (int sidx = 0; sidx < p.splits; ++sidx) {
+              const int4* src = part_ptr(sidx, c);
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                  if (j < nvalid) {
-                    const int4 v = __ldcg(reinterpret_cast<const int4*>(prow + j));
-                    acc[j] += static_cast<uint32_t>(v.x);
-                    acc[j + 1] += static_cast<uint32_t>(v.y);
-                    acc[j + 2] += static_cast<uint32_t>(v.z);
-                    acc[j + 3] += static_cast<uint32_t>(v.w);
-                  }
-                }
+              for (int j = 0; j < 8; ++j) {
+                const int4 v = __ldcg(src + j * 32);
+                acc[4 * j] += static_cast<uint32_t>(v.x);
+                acc[4 * j + 1] += static_cast<uint32_t>(v.y);
+                acc[4 * j + 2] += static_cast<uint32_t>(v.z);
+                acc[4 * j + 3] += static_cast<uint32_t>(v.w);
               }
             }
             float y[32];
@@ -560,30 +582,39 @@ int num_sms() {
 
 struct Plan {
   int bn;
-  int splits;
+  int num_full;      // whole-tile units
+  int tail_tiles;    // tiles split along K
+  int splits;        // parts per tail tile
   int kb_per_split;
 };
 
 constexpr int kPlanSms = 148;  // planning is device-independent so workspace sizes are too
 
+// Tile width: the widest of 256/128/64 whose tile count covers the SMs. Problems with fewer
+// tiles than half the SMs (small M) split every tile along K into S parts whose exact int32
+// partials meet in the workspace. (Splitting only the tiles of a last partial wave was
+// measured slower on the 2048 x 11008 x 4096 shape, so whole tiles are kept there.)
+// LLM.int8 (outlier operands) tiles are never split.
 Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool outliers) {
   const int64_t m_t = (M + kBM - 1) / kBM;
   const int64_t kb = (K + kBK - 1) / kBK;
   auto tiles = [&](int bn) { return m_t * ((N + bn - 1) / bn); };
-  Plan pl{64, 1, static_cast<int>(kb)};
+  Plan pl{64, 0, 0, 1, static_cast<int>(kb)};
   if (tiles(256) >= kPlanSms) {
     pl.bn = 256;
   } else if (tiles(128) >= kPlanSms) {
     pl.bn = 128;
-  } else if (!outliers) {
-    const int64_t base = tiles(64);
-    if (2 * base <= kPlanSms && kb >= 4) {
-      int64_t sp = std::min<int64_t>({kPlanSms / base, kb / 2, 16});
-      const int64_t per = (kb + sp - 1) / sp;
-      pl.splits = static_cast<int>((kb + per - 1) / per);
-      pl.kb_per_split = static_cast<int>(per);
-    }
   }
+  const int64_t T = tiles(pl.bn);
+  pl.num_full = static_cast<int>(T);
+  if (outliers || 2 * T > kPlanSms || kb < 4) return pl;
+  const int64_t S = std::min<int64_t>({kPlanSms / T, kb / 2, 16});
+  if (S < 2) return pl;
+  const int64_t per = (kb + S - 1) / S;
+  pl.splits = static_cast<int>((kb + per - 1) / per);
+  pl.kb_per_split = static_cast<int>(per);
+  pl.tail_tiles = static_cast<int>(T);
+  pl.num_full = 0;
   return pl;
 }
 
@@ -639,21 +670,22 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   p.num_m_tiles = static_cast<int>((a.M + kBM - 1) / kBM);
   p.num_n_tiles = static_cast<int>((a.N + BN - 1) / BN);
   p.num_kb = static_cast<int>((a.K + kBK - 1) / kBK);
+  p.num_full = pl.num_full;
   p.splits = pl.splits;
   p.kb_per_split = pl.kb_per_split;
+  p.num_units = pl.num_full + pl.tail_tiles * pl.splits;
   p.partials = nullptr;
   p.counters = nullptr;
-  if (pl.splits > 1) {
+  if (pl.tail_tiles > 0) {
     p.partials = static_cast<int32_t*>(a.ws);
     p.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(a.ws) +
-                                            up256(sizeof(int32_t) * pl.splits * a.M * a.N));
+                                            up256(sizeof(int32_t) * pl.tail_tiles * pl.splits * kBM * BN));
   }
   p.o_count = a.o_count;
   p.status = device_status_word();
   p.wait_limit_ns = a.wait_limit_ns;
   p.fault = a.fault;
-  const int tiles = p.num_m_tiles * p.num_n_tiles * p.splits;
-  const int grid = std::min(tiles, num_sms());
+  const int grid = std::min(p.num_units, num_sms());
   note_launch();
   w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS><<<grid, kThreads, C::kSmemBytes, stream>>>(tmA, tmB, tmXo, tmWo, tmY, p);
   return cudaGetLastError();
@@ -663,9 +695,9 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, bool outliers) {
   const Plan pl = plan_gemm(M, N, K, outliers);
-  if (pl.splits == 1) return 0;
-  const int64_t tiles_mn = ((M + kBM - 1) / kBM) * ((N + pl.bn - 1) / pl.bn);
-  return up256(sizeof(int32_t) * pl.splits * M * N) + up256(sizeof(int32_t) * tiles_mn * kEpiWarps);
+  if (pl.tail_tiles == 0) return 0;
+  return up256(sizeof(int32_t) * pl.tail_tiles * pl.splits * kBM * pl.bn) +
+         up256(sizeof(int32_t) * pl.tail_tiles * kEpiWarps);
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream, const char** why) {

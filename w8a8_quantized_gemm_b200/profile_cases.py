@@ -1,0 +1,68 @@
+"""Small, self-contained launches of single kernels for profiler captures (ncu).
+
+Usage: python -m w8a8_quantized_gemm_b200.profile_cases {gemm,decode,llm,quant,absmax}
+
+Each case makes random device inputs of one workload's shape and calls one entry point three
+times (so that a capture can skip the first, cold launch):
+  gemm    sq_int8_gemm_dequant, 2048 x 11008 x 4096 (Llama-2-7B MLP up-projection)
+  decode  sq_int8_gemm_dequant, 64 x 4096 x 4096 (decode, split K)
+  llm     llmint8_decomposed_linear, 2048 x 11008 x 4096 with 4 outlier columns
+  quant   sq_quant_act_per_token with smoothing, X bf16 [8192, 8192] (inputs larger than L2)
+  absmax  sq_act_channel_absmax, X bf16 [8192, 8192]
+"""
+import sys
+
+import torch
+
+from w8a8_quantized_gemm_b200 import sq
+
+
+def main(mode: str) -> None:
+    torch.cuda.set_device(0)
+    dev = "cuda"
+    torch.manual_seed(0)
+    if mode in ("gemm", "decode"):
+        M, N, K = (2048, 11008, 4096) if mode == "gemm" else (64, 4096, 4096)
+        Xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev)
+        Wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev)
+        d = torch.rand(M, device=dev) * 1e-2
+        e = torch.rand(N, device=dev) * 1e-3
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = sq.workspace(sq.SQ_OP_INT8_GEMM_DEQUANT, M, N, K)
+        for _ in range(3):
+            sq.sq_int8_gemm_dequant(Xq, Wq, d, e, sq.SQ_PER_CHANNEL, None, Y, None, ws)
+    elif mode == "llm":
+        M, N, K = 2048, 11008, 4096
+        X = torch.randn(M, K, device=dev)
+        X[:, :4] += 50
+        X = X.to(torch.bfloat16)
+        W = (torch.randn(N, K, device=dev) * 0.02).to(torch.bfloat16)
+        Wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+        e = torch.empty(N, device=dev)
+        sq.sq_smooth_quant_weight(W, None, sq.SQ_PER_CHANNEL, Wq, e)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = sq.workspace(sq.SQ_OP_LLMINT8, M, N, K)
+        for _ in range(3):
+            sq.llmint8_decomposed_linear(X, W, Wq, e, 6.0, None, Y, None, None, None, ws)
+    elif mode in ("quant", "absmax"):
+        M, K = 8192, 8192
+        X = torch.randn(M, K, device=dev).to(torch.bfloat16)
+        if mode == "quant":
+            Xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+            dd = torch.empty(M, device=dev)
+            inv = torch.rand(K, device=dev) + 0.5
+            for _ in range(3):
+                sq.sq_quant_act_per_token(X, inv, Xq, dd)
+        else:
+            amax = torch.empty(K, device=dev)
+            for _ in range(3):
+                sq.sq_act_channel_absmax(X, amax)
+    else:
+        raise SystemExit(f"unknown case {mode!r}")
+    sq.sq_sync_status()
+    torch.cuda.synchronize()
+    print("ok", mode)
+
+
+if __name__ == "__main__":
+    main(sys.argv[1] if len(sys.argv) > 1 else "gemm")

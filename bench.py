@@ -142,20 +142,31 @@ def _init_pg(ws, local):
     return ws > 1
 
 
-def _max_over_ranks(x: float, use_dist: bool, local: int) -> float:
+def _max_over_ranks(x: float, use_dist: bool, local) -> float:
+    """Maximum of x over the ranks (x itself on one rank). `local` is the CUDA device index
+    (NCCL) or None for a CPU process group (gloo)."""
     if not use_dist:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device=f"cuda:{local}")
+    t = torch.tensor([x], dtype=torch.float64, device="cpu" if local is None else f"cuda:{local}")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def _barrier(use_dist: bool, local: int):
+def _barrier(use_dist: bool, local):
     if use_dist:
         import torch.distributed as dist
-        dist.barrier(device_ids=[local])
+        if local is None:
+            dist.barrier()
+        else:
+            dist.barrier(device_ids=[local])
+
+
+def whole_job_rate(units_per_step: float, steps: int, world: int, ms_max: float) -> float:
+    """Units per second of the whole job: every rank processed `steps` steps of its own replica
+    in at most `ms_max` milliseconds (the slowest rank's time)."""
+    return units_per_step * world * steps / (ms_max * 1e-3)
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -305,7 +316,7 @@ def run_ours(args):
     del graph
 
     ms_step = ms_total / args.steps
-    value = ops_step * ws * args.steps / (ms_total * 1e-3) / 1e12
+    value = whole_job_rate(ops_step, args.steps, ws, ms_total) / 1e12
 
     # ---------------------------------------------------------------- kernel rooflines
     gemm_ms = per_kernel["int8_gemm_dequant"]
@@ -393,7 +404,7 @@ def run_e2e(path, p, args, ops_step, use_dist, local, ws):
     ms = _max_over_ranks(a.elapsed_time(b), use_dist, local)
     bi = hX.numel() * 2 + hW.numel() * 2
     bo = hY.numel() * 2 + hY2.numel() * 2
-    return {"value": round(ops_step * ws * steps / (ms * 1e-3) / 1e12, 3), "unit": "TOPS",
+    return {"value": round(whole_job_rate(ops_step, steps, ws, ms) / 1e12, 3), "unit": "TOPS",
             "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "steps": steps,
             "ms_per_step": round(ms / steps, 3)}
 

@@ -374,39 +374,65 @@ def run_ours(args):
 
 
 def run_e2e(path, p, args, ops_step, use_dist, local, ws):
-    """Same step through the C ABI with the inputs in pinned HOST memory: H2D of X and W,
-    the step, D2H of both outputs, all inside the timed region."""
+    """Same step through the C ABI with the inputs in pinned HOST memory: every step copies its
+    X and W host-to-device and both outputs device-to-host, all inside the timed region. The
+    copies run on their own streams, so step i's outputs go back and step i+1's inputs come in
+    while step i+1 computes (inputs in the rotating device sets, outputs double-buffered)."""
     import torch
     steps = max(3, min(args.steps, args.e2e_steps))
     hX = torch.from_numpy(np.ascontiguousarray(p.X).view(np.int16)).view(torch.bfloat16).pin_memory()
     hW = torch.from_numpy(np.ascontiguousarray(p.W).view(np.int16)).view(torch.bfloat16).pin_memory()
-    hY = torch.empty(path.Y.shape, dtype=torch.bfloat16).pin_memory()
-    hY2 = torch.empty(path.Y2.shape, dtype=torch.bfloat16).pin_memory()
+    hY = [torch.empty(path.Y.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    hY2 = [torch.empty(path.Y2.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    dY = [path.Y, torch.empty_like(path.Y)]
+    dY2 = [path.Y2, torch.empty_like(path.Y2)]
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    nsets = len(path.X)
 
-    def one(i):
-        k = i % len(path.X)
-        path.X[k].copy_(hX, non_blocking=True)
-        path.W[k].copy_(hW, non_blocking=True)
-        path.step(k)
-        hY.copy_(path.Y, non_blocking=True)
-        hY2.copy_(path.Y2, non_blocking=True)
+    def run(n):
+        ev_in, ev_comp, ev_out = {}, {}, {}
+        for i in range(n):
+            k, b = i % nsets, i % 2
+            with torch.cuda.stream(s_in):
+                if i >= nsets:
+                    s_in.wait_event(ev_comp[i - nsets])  # set k no longer in use
+                path.X[k].copy_(hX, non_blocking=True)
+                path.W[k].copy_(hW, non_blocking=True)
+                ev_in[i] = torch.cuda.Event()
+                ev_in[i].record()
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(ev_in[i])
+                if i >= 2:
+                    s_comp.wait_event(ev_out[i - 2])  # output buffers b copied out
+                path.Y, path.Y2 = dY[b], dY2[b]
+                path.step(k)
+                ev_comp[i] = torch.cuda.Event()
+                ev_comp[i].record()
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[i])
+                hY[b].copy_(dY[b], non_blocking=True)
+                hY2[b].copy_(dY2[b], non_blocking=True)
+                ev_out[i] = torch.cuda.Event()
+                ev_out[i].record()
 
-    for i in range(2):
-        one(i)
+    run(2)
     torch.cuda.synchronize()
     _barrier(use_dist, local)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for i in range(steps):
-        one(i)
-    b.record()
+    a.record(s_in)
+    run(steps)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_comp)
+    b.record(s_out)
     torch.cuda.synchronize()
+    path.Y, path.Y2 = dY[0], dY2[0]
     ms = _max_over_ranks(a.elapsed_time(b), use_dist, local)
     bi = hX.numel() * 2 + hW.numel() * 2
-    bo = hY.numel() * 2 + hY2.numel() * 2
+    bo = hY[0].numel() * 2 + hY2[0].numel() * 2
     return {"value": round(whole_job_rate(ops_step, steps, ws, ms) / 1e12, 3), "unit": "TOPS",
             "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "steps": steps,
-            "ms_per_step": round(ms / steps, 3)}
+            "ms_per_step": round(ms / steps, 3),
+            "mode": "copy-in / compute / copy-out on three streams, overlapped across steps"}
 
 
 # ----------------------------------------------------------------------------- oracle on the host

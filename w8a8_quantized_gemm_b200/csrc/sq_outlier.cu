@@ -14,7 +14,11 @@ namespace {
 constexpr int kMaskThreads = 1024;
 
 // One CTA. Column j is handled by thread j % 1024 of pass j / 1024: a warp covers one
-// 32-column mask word, so the ballot is the word and the scan runs over warps.
+// 32-column mask word, so the ballot is the word and the scan runs over warps. The flags of
+// the first kPrefetch passes are computed from loads issued before the scan loop (one memory
+// round trip for K <= 8192).
+constexpr int kPrefetch = 8;
+
 __global__ void __launch_bounds__(kMaskThreads)
 outlier_mask_kernel(const float* __restrict__ amax, int64_t K, float threshold, uint32_t* __restrict__ mask,
                     int32_t* __restrict__ prefix, int32_t* __restrict__ idx, int32_t* __restrict__ count,
@@ -25,11 +29,22 @@ outlier_mask_kernel(const float* __restrict__ amax, int64_t K, float threshold, 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int64_t words = (K + 31) / 32;
+  bool pre[kPrefetch];
+#pragma unroll
+  for (int i = 0; i < kPrefetch; ++i) {
+    const int64_t j = static_cast<int64_t>(i) * kMaskThreads + threadIdx.x;
+    pre[i] = (j < K) && (__ldg(amax + j) > threshold);
+  }
   if (threadIdx.x == 0) running = 0;
   __syncthreads();
-  for (int64_t base = 0; base < K; base += kMaskThreads) {
+  int pass = 0;
+  for (int64_t base = 0; base < K; base += kMaskThreads, ++pass) {
     const int64_t j = base + threadIdx.x;
-    const bool flag = (j < K) && (amax[j] > threshold);
+    bool flag = false;
+#pragma unroll
+    for (int i = 0; i < kPrefetch; ++i)
+      if (i == pass) flag = pre[i];
+    if (pass >= kPrefetch) flag = (j < K) && (__ldg(amax + j) > threshold);
     const uint32_t ballot = __ballot_sync(0xffffffffu, flag);
     if (lane == 0) warp_cnt[warp] = __popc(ballot);
     __syncthreads();
@@ -61,18 +76,28 @@ outlier_mask_kernel(const float* __restrict__ amax, int64_t K, float threshold, 
   }
 }
 
-// dst[r, c] = src[r, idx[c]] for c < count, 0 for count <= c < roundup(count, 64).
+// One thread per row: dst[r, c] = src[r, idx[c]] for c < count, 0 for count <= c <
+// roundup(count, 64), written 8 columns (16 bytes) at a time.
 __global__ void gather_columns_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t ld,
                                       const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
                                       uint16_t* __restrict__ dst, int64_t ld_dst) {
   const int32_t cnt = __ldg(count);
   const int32_t padded = (cnt + 63) & ~63;
-  const int64_t total = rows * static_cast<int64_t>(padded);
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = e / padded;
-    const int32_t c = static_cast<int32_t>(e - r * padded);
-    dst[r * ld_dst + c] = c < cnt ? src[r * ld + __ldg(idx + c)] : static_cast<uint16_t>(0);
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; r < rows;
+       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint16_t* srow = src + r * ld;
+    uint4* drow = reinterpret_cast<uint4*>(dst + r * ld_dst);
+    for (int32_t c0 = 0; c0 < padded; c0 += 8) {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int32_t c = c0 + 2 * i;
+        const uint32_t lo = c < cnt ? srow[__ldg(idx + c)] : 0u;
+        const uint32_t hi = c + 1 < cnt ? srow[__ldg(idx + c + 1)] : 0u;
+        w[i] = lo | (hi << 16);
+      }
+      drow[c0 / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
   }
 }
 
@@ -92,8 +117,9 @@ cudaError_t launch_gather_columns(const uint16_t* src, int64_t rows, int64_t ld,
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t blocks = std::min<int64_t>((rows + 127) / 128, static_cast<int64_t>(sms) * 8);
   note_launch();
-  gather_columns_kernel<<<sms * 4, 256, 0, stream>>>(src, rows, ld, idx, count, dst, ld_dst);
+  gather_columns_kernel<<<static_cast<unsigned>(blocks), 128, 0, stream>>>(src, rows, ld, idx, count, dst, ld_dst);
   return cudaGetLastError();
 }
 

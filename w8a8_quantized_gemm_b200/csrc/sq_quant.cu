@@ -301,15 +301,17 @@ cudaError_t launch_t(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, c
   return cudaGetLastError();
 }
 
-// Shape dispatch: the smallest threads-per-row that keeps <= 32 smoothed values per thread
-// in registers; rows longer than 16384 take the two-read path.
+// Shape dispatch: one 16-element chunk per thread up to K = 4096 (a row over up to 256
+// threads, few registers, several CTAs per SM); longer rows take two chunks per thread, and
+// rows longer than 16384 the two-read path. (Measured: one chunk per thread is faster at
+// K = 4096, two chunks at K = 8192.)
 template <bool OUTLIERS, int MODE>
 cudaError_t dispatch(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, const float* vec,
                      const OutlierView& ov, int8_t* q, float* scale, unsigned int* gmax, cudaStream_t stream) {
   if (K <= 512) return launch_t<32, 1, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
-  if (K <= 1024) return launch_t<32, 2, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
-  if (K <= 2048) return launch_t<64, 2, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
-  if (K <= 4096) return launch_t<128, 2, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
+  if (K <= 1024) return launch_t<64, 1, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
+  if (K <= 2048) return launch_t<128, 1, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
+  if (K <= 4096) return launch_t<256, 1, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
   if (K <= 8192) return launch_t<256, 2, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
   if (K <= 16384) return launch_t<512, 2, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
   return launch_t<512, 1, true, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);

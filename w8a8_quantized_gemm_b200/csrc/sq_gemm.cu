@@ -17,6 +17,10 @@
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one output row per
 //              thread), y = (float(acc) * d_m) * e_n (+ o) (+ bias) -> bf16, global stores;
 //              overlaps the next tile's main loop through the second TMEM buffer.
+// For a few tokens (M <= 64) the operands swap roles: the weight supplies the 128-row MMA
+// operand (output channels on TMEM lanes) and the tokens the N dimension, so no MMA row
+// and no weight byte is spent on padding; the epilogue then applies the per-token scale
+// per column and the per-channel scale and bias per row, and stores transposed boxes.
 // Every mbarrier wait is bounded; on timeout the kernel records an error bit in the
 // device status word, drains its own TMA loads and MMAs, frees TMEM and returns.
 #include "sq_internal.h"
@@ -63,6 +67,9 @@ struct Params {
   const uint16_t* bias;
   int32_t* acc_out;
   int64_t M, N;
+  // Tile space: `rows` along the 128-row MMA operand, `cols` along the BN-column one
+  // (M and N, or N and M when the operands are swapped).
+  int64_t rows, cols;
   int num_m_tiles, num_n_tiles, num_kb;
   // Work units: units [0, num_full) are whole output tiles (tile index = unit); the tiles
   // after them ("tail" tiles) are split along K into `splits` units of kb_per_split k-blocks,
@@ -132,30 +139,45 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // Per-warp column constants of a 32-column chunk, spread over the lanes: lane l holds the
-// weight scales of columns 4*(l%8)..4*(l%8)+3 of chunk l/8 (float4) and their 4 bf16 biases,
+// scales of columns 4*(l%8)..4*(l%8)+3 of chunk l/8 (float4) and their 4 bf16 biases,
 // so a warp covers 4 chunks (128 columns). Loaded before the accumulator is ready.
+// Columns are output channels (weight scale, bias) or, with swapped operands, tokens
+// (per-token activation scale; the bias then belongs to the row).
 struct ColConsts {
   float4 e;
   uint2 b;
 };
 
+template <bool SWAP>
 __device__ __forceinline__ ColConsts load_col_consts(const Params& p, int64_t n_half0, int lane, int chunks) {
   ColConsts cc;
   const int c = lane >> 3;
   const int64_t n = n_half0 + c * 32 + (lane & 7) * 4;
-  const bool ok = c < chunks && n < p.N;
-  if (p.w_per_channel) {
-    cc.e = ok ? __ldg(reinterpret_cast<const float4*>(p.w_scale + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  const bool ok = c < chunks && n < p.cols;
+  if constexpr (SWAP) {
+    // x_scale has no alignment contract and M need not be a multiple of 4: scalar loads
+    float v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = (ok && n + i < p.cols) ? __ldg(p.x_scale + n + i) : 0.0f;
+    cc.e = make_float4(v[0], v[1], v[2], v[3]);
+    cc.b = make_uint2(0u, 0u);
   } else {
-    const float e0 = __ldg(p.w_scale);
-    cc.e = make_float4(e0, e0, e0, e0);
+    if (p.w_per_channel) {
+      cc.e = ok ? __ldg(reinterpret_cast<const float4*>(p.w_scale + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+      const float e0 = __ldg(p.w_scale);
+      cc.e = make_float4(e0, e0, e0, e0);
+    }
+    cc.b = (p.bias != nullptr && ok) ? __ldg(reinterpret_cast<const uint2*>(p.bias + n)) : make_uint2(0u, 0u);
   }
-  cc.b = (p.bias != nullptr && ok) ? __ldg(reinterpret_cast<const uint2*>(p.bias + n)) : make_uint2(0u, 0u);
   return cc;
 }
 
-// y[j] = (float(acc[j]) * d_m) * e[n0+j] for the 32 columns of chunk c.
-__device__ __forceinline__ void dequant32(const uint32_t (&acc)[32], float d_m, const ColConsts& cc, int c,
+// y[j] = (float(acc[j]) * d_m) * e_n for the 32 columns of chunk c: d_m is the row
+// constant and e_n comes from the lanes' column constants, or, with swapped operands,
+// d_m comes from the column constants and e_n is the row constant.
+template <bool SWAP>
+__device__ __forceinline__ void dequant32(const uint32_t (&acc)[32], float row_scale, const ColConsts& cc, int c,
                                           float (&y)[32]) {
 #pragma unroll
   for (int j = 0; j < 32; j += 4) {
@@ -163,50 +185,94 @@ __device__ __forceinline__ void dequant32(const uint32_t (&acc)[32], float d_m, 
     const float e[4] = {__shfl_sync(0xffffffffu, cc.e.x, src), __shfl_sync(0xffffffffu, cc.e.y, src),
                         __shfl_sync(0xffffffffu, cc.e.z, src), __shfl_sync(0xffffffffu, cc.e.w, src)};
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      y[j + u] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(acc[j + u])), d_m), e[u]);
+    for (int u = 0; u < 4; ++u) {
+      const float a = static_cast<float>(static_cast<int32_t>(acc[j + u]));
+      y[j + u] = SWAP ? __fmul_rn(__fmul_rn(a, e[u]), row_scale) : __fmul_rn(__fmul_rn(a, row_scale), e[u]);
+    }
   }
 }
 
-// y[j] += bias[n0+j] (when there is a bias), then pack to bf16 pairs.
+// y[j] += bias (per column, or the row's bias with swapped operands) when there is one,
+// then pack to bf16 pairs.
+template <bool SWAP>
 __device__ __forceinline__ void bias_pack32(float (&y)[32], bool has_bias, const ColConsts& cc, int c,
-                                            uint32_t (&out)[16]) {
+                                            float row_bias, uint32_t (&out)[16]) {
   if (has_bias) {
+    if constexpr (SWAP) {
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-      const int src = c * 8 + j / 4;
-      const uint32_t b0 = __shfl_sync(0xffffffffu, cc.b.x, src);
-      const uint32_t b1 = __shfl_sync(0xffffffffu, cc.b.y, src);
-      y[j] = __fadd_rn(y[j], __uint_as_float(b0 << 16));
-      y[j + 1] = __fadd_rn(y[j + 1], __uint_as_float(b0 & 0xFFFF0000u));
-      y[j + 2] = __fadd_rn(y[j + 2], __uint_as_float(b1 << 16));
-      y[j + 3] = __fadd_rn(y[j + 3], __uint_as_float(b1 & 0xFFFF0000u));
+      for (int j = 0; j < 32; ++j) y[j] = __fadd_rn(y[j], row_bias);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const int src = c * 8 + j / 4;
+        const uint32_t b0 = __shfl_sync(0xffffffffu, cc.b.x, src);
+        const uint32_t b1 = __shfl_sync(0xffffffffu, cc.b.y, src);
+        y[j] = __fadd_rn(y[j], __uint_as_float(b0 << 16));
+        y[j + 1] = __fadd_rn(y[j + 1], __uint_as_float(b0 & 0xFFFF0000u));
+        y[j + 2] = __fadd_rn(y[j + 2], __uint_as_float(b1 << 16));
+        y[j + 3] = __fadd_rn(y[j + 3], __uint_as_float(b1 & 0xFFFF0000u));
+      }
     }
   }
 #pragma unroll
   for (int j = 0; j < 16; ++j) out[j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
 }
 
-// One 32x32 bf16 box (this lane's row, 32 columns) through the warp's staging buffer to a
-// TMA store at (n0, row0).
+// Debug copy of the int32 accumulators of one 32-column chunk (nvalid valid columns) of
+// tile row r; with swapped operands the row is output channel r and the columns tokens.
+template <bool SWAP>
+__device__ __forceinline__ void store_acc32(const Params& p, const uint32_t (&acc)[32], int64_t r, int64_t n0,
+                                            int nvalid) {
+  if constexpr (SWAP) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < nvalid) p.acc_out[(n0 + j) * p.N + r] = static_cast<int32_t>(acc[j]);
+  } else {
+    int32_t* arow = p.acc_out + r * p.N + n0;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      if (j < nvalid) *reinterpret_cast<uint4*>(arow + j) = make_uint4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+    }
+  }
+}
+
+// One 32x32 bf16 box through the warp's staging buffer to a TMA store. Each lane holds
+// 32 values of its tile row. Normally the row is an output row: the box is stored at
+// (column n0, row row0) with one staging row per lane. With swapped operands the lane's
+// row is an output channel, so lane l writes staging column l of 32 token rows and the
+// box goes to (channel row0, token n0).
+template <bool SWAP>
 __device__ __forceinline__ void store_box(const uint32_t (&v)[16], uint8_t* stage_tiles, int& ebuf, int lane,
                                           const CUtensorMap* tmY, int64_t n0, int64_t row0) {
   // staging buffer `ebuf` was last read by the TMA store issued two boxes ago
   if (lane == 0) bulk_wait_group_read<kEpiBufs - 1>();
   __syncwarp();
-  uint4* st = reinterpret_cast<uint4*>(stage_tiles + ebuf * kStageTileBytes + lane * 64);
+  uint8_t* tile = stage_tiles + ebuf * kStageTileBytes;
+  if constexpr (SWAP) {
+    uint16_t* st = reinterpret_cast<uint16_t*>(tile) + lane;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) st[j] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    for (int j = 0; j < 16; ++j) {
+      st[(2 * j) * 32] = static_cast<uint16_t>(v[j] & 0xFFFFu);
+      st[(2 * j + 1) * 32] = static_cast<uint16_t>(v[j] >> 16);
+    }
+  } else {
+    uint4* st = reinterpret_cast<uint4*>(tile + lane * 64);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) st[j] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  }
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
-    tma_store_2d(tmY, stage_tiles + ebuf * kStageTileBytes, static_cast<int32_t>(n0), static_cast<int32_t>(row0));
+    if constexpr (SWAP)
+      tma_store_2d(tmY, tile, static_cast<int32_t>(row0), static_cast<int32_t>(n0));
+    else
+      tma_store_2d(tmY, tile, static_cast<int32_t>(n0), static_cast<int32_t>(row0));
     bulk_commit_group();
   }
   ebuf ^= 1;
 }
 
-template <int BN, bool OUTLIERS, int ACC_BUFS>
+template <int BN, bool OUTLIERS, int ACC_BUFS, bool SWAP>
 __global__ void __launch_bounds__(kThreads, 1)
 w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmXo, const __grid_constant__ CUtensorMap tmWo,
@@ -377,6 +443,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     // to the MMA warp before the stores; each 32x32 bf16 box then goes through this warp's
     // staging buffer in shared memory to a TMA store.
     constexpr int kChunks = BN / 64;  // 32-column chunks per warp
+    static_assert(!(SWAP && OUTLIERS), "swapped operands carry no outlier product");
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
@@ -391,11 +458,21 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const int tile_mn = w.tile_mn;
       const int split = w.split;
       const int64_t m_tile0 = static_cast<int64_t>(tile_mn % p.num_m_tiles) * kBM;
-      const int64_t m = m_tile0 + row;
+      const int64_t r = m_tile0 + row;  // this thread's tile row (output row, or channel if swapped)
+      const int64_t box_row0 = m_tile0 + quad * 32;
+      const bool rows_live = box_row0 < p.rows;  // uniform across the warp
       const int64_t n_half0 = static_cast<int64_t>(tile_mn / p.num_m_tiles) * BN + half * (BN / 2);
-      const bool m_ok = m < p.M;
-      const float d_m = m_ok ? __ldg(p.x_scale + m) : 0.0f;
-      const ColConsts cc = load_col_consts(p, n_half0, lane, kChunks);
+      const bool r_ok = r < p.rows;
+      float row_scale = 0.0f, row_bias = 0.0f;
+      if constexpr (SWAP) {
+        if (r_ok) {
+          row_scale = __ldg(p.w_scale + (p.w_per_channel ? r : 0));
+          if (p.bias != nullptr) row_bias = __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + r)) << 16);
+        }
+      } else {
+        row_scale = r_ok ? __ldg(p.x_scale + r) : 0.0f;
+      }
+      const ColConsts cc = load_col_consts<SWAP>(p, n_half0, lane, kChunks);
       const bool has_bias = p.bias != nullptr;
       // lane 0 waits and the warp follows its verdict, so the warp stays converged
       int ok = 0;
@@ -413,22 +490,15 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
           const int64_t n0 = n_half0 + c * 32;
-          if (n0 < p.N) {  // uniform across the warp
+          if (n0 < p.cols) {  // uniform across the warp
             __syncwarp();
             uint32_t acc[32];
             tmem_ld_32x32b_x32(t_row + c * 32, acc);
             tmem_wait_ld();
-            const int nvalid = (p.N - n0) < 32 ? static_cast<int>(p.N - n0) : 32;  // a multiple of 8
+            const int nvalid = (p.cols - n0) < 32 ? static_cast<int>(p.cols - n0) : 32;
             float y[32];
-            dequant32(acc, d_m, cc, c, y);
-            if (p.acc_out != nullptr && m_ok) {
-              int32_t* arow = p.acc_out + m * p.N + n0;
-#pragma unroll
-              for (int j = 0; j < 32; j += 4) {
-                if (j < nvalid)
-                  *reinterpret_cast<uint4*>(arow + j) = make_uint4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-              }
-            }
+            dequant32<SWAP>(acc, row_scale, cc, c, y);
+            if (p.acc_out != nullptr && r_ok) store_acc32<SWAP>(p, acc, r, n0, nvalid);
             if constexpr (OUTLIERS) {
               if (kb_o > 0) {
                 uint32_t of[32];  // fp32 outlier product of the same 32 columns
@@ -438,17 +508,19 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 for (int j = 0; j < 32; ++j) y[j] = __fadd_rn(y[j], __uint_as_float(of[j]));
               }
             }
-            bias_pack32(y, has_bias, cc, c, packed[c]);
+            bias_pack32<SWAP>(y, has_bias, cc, c, row_bias, packed[c]);
           }
         }
         // the accumulator is no longer needed: hand it back before storing
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(tmem_empty + buf);
+        if (rows_live) {
 #pragma unroll
-        for (int c = 0; c < kChunks; ++c) {
-          const int64_t n0 = n_half0 + c * 32;
-          if (n0 < p.N) store_box(packed[c], stage_tiles, ebuf, lane, &tmY, n0, m_tile0 + quad * 32);
+          for (int c = 0; c < kChunks; ++c) {
+            const int64_t n0 = n_half0 + c * 32;
+            if (n0 < p.cols) store_box<SWAP>(packed[c], stage_tiles, ebuf, lane, &tmY, n0, box_row0);
+          }
         }
       } else {
         // K split: this split's int32 partial goes to the workspace; the warp that brings
@@ -463,7 +535,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
           const int64_t n0 = n_half0 + c * 32;
-          if (n0 < p.N) {
+          if (n0 < p.cols) {
             __syncwarp();
             uint32_t acc[32];
             tmem_ld_32x32b_x32(t_row + c * 32, acc);
@@ -488,13 +560,13 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           }
         }
         last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
+        if (last && rows_live) {
           __threadfence();
 #pragma unroll 1
           for (int c = 0; c < kChunks; ++c) {
             const int64_t n0 = n_half0 + c * 32;
-            if (n0 >= p.N) break;
-            const int nvalid = (p.N - n0) < 32 ? static_cast<int>(p.N - n0) : 32;
+            if (n0 >= p.cols) break;
+            const int nvalid = (p.cols - n0) < 32 ? static_cast<int>(p.cols - n0) : 32;
             uint32_t acc[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) acc[j] = 0;
@@ -510,18 +582,11 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
               }
             }
             float y[32];
-            dequant32(acc, d_m, cc, c, y);
-            if (p.acc_out != nullptr && m_ok) {
-              int32_t* arow = p.acc_out + m * p.N + n0;
-#pragma unroll
-              for (int j = 0; j < 32; j += 4) {
-                if (j < nvalid)
-                  *reinterpret_cast<uint4*>(arow + j) = make_uint4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-              }
-            }
+            dequant32<SWAP>(acc, row_scale, cc, c, y);
+            if (p.acc_out != nullptr && r_ok) store_acc32<SWAP>(p, acc, r, n0, nvalid);
             uint32_t packed[16];
-            bias_pack32(y, has_bias, cc, c, packed);
-            store_box(packed, stage_tiles, ebuf, lane, &tmY, n0, m_tile0 + quad * 32);
+            bias_pack32<SWAP>(y, has_bias, cc, c, row_bias, packed);
+            store_box<SWAP>(packed, stage_tiles, ebuf, lane, &tmY, n0, box_row0);
           }
         }
       }
@@ -581,6 +646,7 @@ int num_sms() {
 }
 
 struct Plan {
+  bool swap;         // weight rows on the 128-row MMA operand, tokens on the BN columns
   int bn;
   int num_full;      // whole-tile units
   int tail_tiles;    // tiles split along K
@@ -590,17 +656,26 @@ struct Plan {
 
 constexpr int kPlanSms = 148;  // planning is device-independent so workspace sizes are too
 
-// Tile width: the widest of 256/128/64 whose tile count covers the SMs. Problems with fewer
-// tiles than half the SMs (small M) split every tile along K into S parts whose exact int32
-// partials meet in the workspace. (Splitting only the tiles of a last partial wave was
-// measured slower on the 2048 x 11008 x 4096 shape, so whole tiles are kept there.)
-// LLM.int8 (outlier operands) tiles are never split.
+constexpr int64_t kSwapMaxM = 64;  // token counts that fit one 64-column tile
+
+// Operand roles: up to 64 tokens (and no outlier product) swap the operands, so the weight
+// rows fill the 128-row MMA operand and the tokens one 64-column tile. Otherwise the tile
+// width is the widest of 256/128/64 whose tile count covers the SMs. Problems with fewer
+// tiles than half the SMs (small M, or a swapped decode shape) split every tile along K
+// into S parts whose exact int32 partials meet in the workspace. (Splitting only the tiles
+// of a last partial wave was measured slower on the 2048 x 11008 x 4096 shape, so whole
+// tiles are kept there.) LLM.int8 (outlier operands) tiles are never split.
 Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool outliers) {
-  const int64_t m_t = (M + kBM - 1) / kBM;
+  const bool swap = !outliers && M <= kSwapMaxM;
+  const int64_t rows = swap ? N : M;
+  const int64_t cols = swap ? M : N;
+  const int64_t m_t = (rows + kBM - 1) / kBM;
   const int64_t kb = (K + kBK - 1) / kBK;
-  auto tiles = [&](int bn) { return m_t * ((N + bn - 1) / bn); };
-  Plan pl{64, 0, 0, 1, static_cast<int>(kb)};
-  if (tiles(256) >= kPlanSms) {
+  auto tiles = [&](int bn) { return m_t * ((cols + bn - 1) / bn); };
+  Plan pl{swap, 64, 0, 0, 1, static_cast<int>(kb)};
+  if (swap) {
+    pl.bn = 64;
+  } else if (tiles(256) >= kPlanSms) {
     pl.bn = 256;
   } else if (tiles(128) >= kPlanSms) {
     pl.bn = 128;
@@ -620,13 +695,18 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool outliers) {
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
-template <int BN, bool OUTLIERS, int ACC_BUFS>
+template <int BN, bool OUTLIERS, int ACC_BUFS, bool SWAP>
 cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const char** why) {
   using C = Cfg<BN, OUTLIERS, ACC_BUFS>;
   CUtensorMap tmA{}, tmB{}, tmXo{}, tmWo{}, tmY{};
   const uint64_t K = static_cast<uint64_t>(a.K);
-  if (!make_operand_map(&tmA, a.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, a.M, K, kBM) ||
-      !make_operand_map(&tmB, a.Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, a.N, K, BN)) {
+  // A: the 128-row operand (Xq, or Wq when swapped); B: the BN-row operand
+  const int8_t* a_ptr = SWAP ? a.Wq : a.Xq;
+  const int8_t* b_ptr = SWAP ? a.Xq : a.Wq;
+  const int64_t rows = SWAP ? a.N : a.M;
+  const int64_t cols = SWAP ? a.M : a.N;
+  if (!make_operand_map(&tmA, a_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, rows, K, kBM) ||
+      !make_operand_map(&tmB, b_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, cols, K, BN)) {
     *why = "cuTensorMapEncodeTiled failed for the int8 operands";
     return cudaErrorInvalidValue;
   }
@@ -651,7 +731,7 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   cudaGetDevice(&dev);
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_done.load() & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS>,
+    cudaError_t e = cudaFuncSetAttribute(w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS, SWAP>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) {
       *why = "cudaFuncSetAttribute(MaxDynamicSharedMemorySize) failed";
@@ -667,8 +747,10 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   p.acc_out = a.acc_out;
   p.M = a.M;
   p.N = a.N;
-  p.num_m_tiles = static_cast<int>((a.M + kBM - 1) / kBM);
-  p.num_n_tiles = static_cast<int>((a.N + BN - 1) / BN);
+  p.rows = rows;
+  p.cols = cols;
+  p.num_m_tiles = static_cast<int>((rows + kBM - 1) / kBM);
+  p.num_n_tiles = static_cast<int>((cols + BN - 1) / BN);
   p.num_kb = static_cast<int>((a.K + kBK - 1) / kBK);
   p.num_full = pl.num_full;
   p.splits = pl.splits;
@@ -687,7 +769,7 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   p.fault = a.fault;
   const int grid = std::min(p.num_units, num_sms());
   note_launch();
-  w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS><<<grid, kThreads, C::kSmemBytes, stream>>>(tmA, tmB, tmXo, tmWo, tmY, p);
+  w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS, SWAP><<<grid, kThreads, C::kSmemBytes, stream>>>(tmA, tmB, tmXo, tmWo, tmY, p);
   return cudaGetLastError();
 }
 
@@ -705,13 +787,14 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream, const char** why
   const Plan pl = plan_gemm(a.M, a.N, a.K, outliers);
   if (outliers) {
     // int32 + fp32 accumulators: 256-wide tiles fit TMEM once, narrower ones twice
-    if (pl.bn == 256) return run<256, true, 1>(a, pl, stream, why);
-    if (pl.bn == 128) return run<128, true, 2>(a, pl, stream, why);
-    return run<64, true, 2>(a, pl, stream, why);
+    if (pl.bn == 256) return run<256, true, 1, false>(a, pl, stream, why);
+    if (pl.bn == 128) return run<128, true, 2, false>(a, pl, stream, why);
+    return run<64, true, 2, false>(a, pl, stream, why);
   }
-  if (pl.bn == 256) return run<256, false, 2>(a, pl, stream, why);
-  if (pl.bn == 128) return run<128, false, 2>(a, pl, stream, why);
-  return run<64, false, 2>(a, pl, stream, why);
+  if (pl.swap) return run<64, false, 2, true>(a, pl, stream, why);
+  if (pl.bn == 256) return run<256, false, 2, false>(a, pl, stream, why);
+  if (pl.bn == 128) return run<128, false, 2, false>(a, pl, stream, why);
+  return run<64, false, 2, false>(a, pl, stream, why);
 }
 
 }  // namespace sq

@@ -324,6 +324,9 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // set-up done: from here on global memory written by the previous kernel is read
+  griddep_wait();
+  griddep_launch_dependents();
 
   const int num_units = p.num_units;
   int kb_o = 0;
@@ -768,9 +771,11 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   p.wait_limit_ns = a.wait_limit_ns;
   p.fault = a.fault;
   const int grid = std::min(p.num_units, num_sms());
-  note_launch();
-  w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS, SWAP><<<grid, kThreads, C::kSmemBytes, stream>>>(tmA, tmB, tmXo, tmWo, tmY, p);
-  return cudaGetLastError();
+  // short, latency-bound launches (swapped or K-split plans) overlap their set-up with
+  // the previous kernel's tail
+  const bool programmatic = SWAP || pl.tail_tiles > 0;
+  return launch_kernel(w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS, SWAP>, dim3(grid), dim3(kThreads), C::kSmemBytes,
+                       stream, programmatic, tmA, tmB, tmXo, tmWo, tmY, p);
 }
 
 }  // namespace

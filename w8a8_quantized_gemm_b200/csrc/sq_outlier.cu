@@ -26,6 +26,8 @@ outlier_mask_kernel(const float* __restrict__ amax, int64_t K, float threshold, 
   __shared__ int32_t warp_cnt[kMaskThreads / 32];
   __shared__ int32_t warp_off[kMaskThreads / 32];
   __shared__ int32_t running;
+  griddep_wait();
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int64_t words = (K + 31) / 32;
@@ -81,6 +83,8 @@ outlier_mask_kernel(const float* __restrict__ amax, int64_t K, float threshold, 
 __global__ void gather_columns_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t ld,
                                       const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
                                       uint16_t* __restrict__ dst, int64_t ld_dst) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int32_t cnt = __ldg(count);
   const int32_t padded = (cnt + 63) & ~63;
   for (int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; r < rows;
@@ -106,10 +110,8 @@ __global__ void gather_columns_kernel(const uint16_t* __restrict__ src, int64_t 
 cudaError_t launch_outlier_mask(const float* amax, int64_t K, float threshold, uint32_t* mask, int32_t* prefix,
                                 int32_t* idx, int32_t* count, uint32_t* mask_out, int32_t* count_out,
                                 cudaStream_t stream) {
-  note_launch();
-  outlier_mask_kernel<<<1, kMaskThreads, 0, stream>>>(amax, K, threshold, mask, prefix, idx, count, mask_out,
-                                                       count_out);
-  return cudaGetLastError();
+  return launch_kernel(outlier_mask_kernel, dim3(1), dim3(kMaskThreads), 0, stream, false, amax, K, threshold,
+                       mask, prefix, idx, count, mask_out, count_out);
 }
 
 cudaError_t launch_gather_columns(const uint16_t* src, int64_t rows, int64_t ld, const int32_t* idx,
@@ -118,9 +120,8 @@ cudaError_t launch_gather_columns(const uint16_t* src, int64_t rows, int64_t ld,
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t blocks = std::min<int64_t>((rows + 127) / 128, static_cast<int64_t>(sms) * 8);
-  note_launch();
-  gather_columns_kernel<<<static_cast<unsigned>(blocks), 128, 0, stream>>>(src, rows, ld, idx, count, dst, ld_dst);
-  return cudaGetLastError();
+  return launch_kernel(gather_columns_kernel, dim3(static_cast<unsigned>(blocks)), dim3(128), 0, stream, false,
+                       src, rows, ld, idx, count, dst, ld_dst);
 }
 
 }  // namespace sq

@@ -123,6 +123,8 @@ quant_rows_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
                   const float* __restrict__ vec, OutlierView ov, int8_t* __restrict__ q,
                   float* __restrict__ scale, unsigned int* __restrict__ gmax_bits) {
   constexpr int kThreads = TPR > kCta ? TPR : kCta;
+  griddep_wait();
+  griddep_launch_dependents();
   constexpr int kGroups = kThreads / TPR;
   constexpr int kVC = (HAS_VEC && !TWO_PASS) ? CHUNKS : 1;
   __shared__ float red[kThreads / 32];
@@ -286,19 +288,18 @@ cudaError_t launch_t(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, c
   constexpr int kThreads = TPR > kCta ? TPR : kCta;
   constexpr int kGroups = kThreads / TPR;
   const int64_t groups = (rows + kGroups - 1) / kGroups;
-  note_launch();
   if (vec != nullptr) {
     static int per_sm = 0;
     auto kernel = quant_rows_kernel<TPR, CHUNKS, TWO_PASS, OUTLIERS, true, MODE>;
     const int64_t blocks = resident_grid(kernel, kThreads, groups, per_sm);
-    kernel<<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(src, rows, K, ld, vec, ov, q, scale, gmax);
-  } else {
-    static int per_sm = 0;
-    auto kernel = quant_rows_kernel<TPR, CHUNKS, TWO_PASS, OUTLIERS, false, MODE>;
-    const int64_t blocks = resident_grid(kernel, kThreads, groups, per_sm);
-    kernel<<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(src, rows, K, ld, vec, ov, q, scale, gmax);
+    return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, stream, false, src, rows,
+                         K, ld, vec, ov, q, scale, gmax);
   }
-  return cudaGetLastError();
+  static int per_sm = 0;
+  auto kernel = quant_rows_kernel<TPR, CHUNKS, TWO_PASS, OUTLIERS, false, MODE>;
+  const int64_t blocks = resident_grid(kernel, kThreads, groups, per_sm);
+  return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, stream, false, src, rows, K,
+                       ld, vec, ov, q, scale, gmax);
 }
 
 // Shape dispatch: one 16-element chunk per thread up to K = 4096 (a row over up to 256
@@ -327,7 +328,7 @@ cudaError_t launch_quant_rows(const uint16_t* src, int64_t rows, int64_t K, int6
 
 cudaError_t launch_quant_tensor(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, const float* vec,
                                 unsigned int* gmax_bits, int8_t* q, float* scale1, cudaStream_t stream) {
-  cudaError_t e = cudaMemsetAsync(gmax_bits, 0, sizeof(unsigned int), stream);
+  cudaError_t e = launch_zero_words(gmax_bits, 1, stream);
   if (e != cudaSuccess) return e;
   OutlierView none;
   e = dispatch<false, kTensorMax>(src, rows, K, ld, vec, none, nullptr, nullptr, gmax_bits, stream);

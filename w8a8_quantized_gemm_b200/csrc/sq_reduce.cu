@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(kColWarps * 32)
 col_absmax_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int64_t rows_per_cta,
                   unsigned int* __restrict__ out_bits) {
   __shared__ float part[kColWarps][kColsPerCta];
+  griddep_wait();
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int64_t col0 = static_cast<int64_t>(blockIdx.x) * kColsPerCta + lane * 8;
@@ -83,6 +85,8 @@ col_absmax_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
 // s_j = fp32( pow(max(a_j,1e-8), alpha) / pow(max(w_j,1e-8), 1-alpha) ) in fp64; inv_s = 1/s in fp32.
 __global__ void smooth_factors_kernel(const float* __restrict__ act_amax, float* __restrict__ s_inout,
                                       float* __restrict__ inv_s, int64_t K, float alpha) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (j >= K) return;
   const float a = fmaxf(act_amax[j], 1e-8f);
@@ -94,12 +98,27 @@ __global__ void smooth_factors_kernel(const float* __restrict__ act_amax, float*
   inv_s[j] = __fdiv_rn(1.0f, sj);
 }
 
+__global__ void zero_words_kernel(uint32_t* __restrict__ words, int64_t n) {
+  griddep_wait();
+  griddep_launch_dependents();
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    words[i] = 0u;
+}
+
 }  // namespace
+
+cudaError_t launch_zero_words(uint32_t* words, int64_t n, cudaStream_t stream) {
+  const int threads = 256;
+  const int64_t blocks = std::min<int64_t>(std::max<int64_t>(1, (n + threads - 1) / threads), 1024);
+  return launch_kernel(zero_words_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream, false,
+                       words, n);
+}
 
 cudaError_t launch_col_absmax(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, float* amax,
                               bool accumulate, cudaStream_t stream) {
   if (!accumulate) {
-    cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float) * static_cast<size_t>(K), stream);
+    cudaError_t e = launch_zero_words(reinterpret_cast<uint32_t*>(amax), K, stream);
     if (e != cudaSuccess) return e;
   }
   int dev = 0, sms = 148;
@@ -117,19 +136,16 @@ cudaError_t launch_col_absmax(const uint16_t* src, int64_t rows, int64_t K, int6
     rows_per_cta = (rows + row_blocks - 1) / row_blocks;
   }
   dim3 grid(static_cast<unsigned>(col_blocks), static_cast<unsigned>(row_blocks));
-  note_launch();
-  col_absmax_kernel<<<grid, kColWarps * 32, 0, stream>>>(src, rows, K, ld, rows_per_cta,
-                                                         reinterpret_cast<unsigned int*>(amax));
-  return cudaGetLastError();
+  return launch_kernel(col_absmax_kernel, grid, dim3(kColWarps * 32), 0, stream, false, src, rows, K, ld,
+                       rows_per_cta, reinterpret_cast<unsigned int*>(amax));
 }
 
 cudaError_t launch_smooth_factors(const float* act_amax, float* s_inout, float* inv_s, int64_t K, float alpha,
                                   cudaStream_t stream) {
   const int threads = 256;
   const int64_t blocks = (K + threads - 1) / threads;
-  note_launch();
-  smooth_factors_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(act_amax, s_inout, inv_s, K, alpha);
-  return cudaGetLastError();
+  return launch_kernel(smooth_factors_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream, false,
+                       act_amax, s_inout, inv_s, K, alpha);
 }
 
 }  // namespace sq

@@ -24,6 +24,8 @@ CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off"
 
 PER_TENSOR = 0
 PER_CHANNEL = 1
+NORM_LAYER = 0
+NORM_RMS = 1
 
 
 def build(force: bool = False) -> str:
@@ -52,6 +54,14 @@ def lib():
             "oracle_dequant": ([p, i64, i64, p, p, i32, p, p, p, p], None),
             "oracle_outlier_columns": ([p, i64, f32, p, p, p], C.c_int32),
             "oracle_outlier_product": ([p, i64, p, i64, i64, i64, p, C.c_int32, p], None),
+            "oracle_quant_act_per_tensor": ([p, i64, i64, i64, p, f32, p, p], None),
+            "oracle_smooth_scale_normalize": ([p, p, i64], None),
+            "oracle_norm_smooth_quant": ([p, i64, i64, i64, i32, p, p, f32, p, p, p, p], None),
+            "oracle_mean_std_threshold": ([p, i64, i64, i64, C.c_double, p, p], f32),
+            "oracle_abs_percentile": ([p, i64, i64, i64, C.c_double], f32),
+            "oracle_quant_act_per_token_asym": ([p, i64, i64, i64, p, p, p, p], None),
+            "oracle_weight_row_sums": ([p, i64, i64, p], None),
+            "oracle_dequant_ex": ([p, i64, i64, p, i32, p, i32, p, p, p, p, p], None),
             "oracle_bf16_to_float": ([p, i64, p], None),
             "oracle_float_to_bf16": ([p, i64, p], None),
             "oracle_num_threads": ([], i32),
@@ -98,14 +108,16 @@ def act_channel_absmax(X, prev: Optional[np.ndarray] = None) -> np.ndarray:
     return amax
 
 
-def smooth_scale(act_amax, W, alpha: float):
-    """Returns (s, inv_s), fp32 [K]."""
+def smooth_scale(act_amax, W, alpha: float, normalize: bool = False):
+    """Returns (s, inv_s), fp32 [K]; ``normalize`` applies s/max(s)*127 clamped at 1e-5."""
     a = _c(act_amax, np.float32)
     W = _c(W, np.uint16)
     N, K = W.shape
     s = np.empty(K, np.float32)
     inv_s = np.empty(K, np.float32)
     lib().oracle_smooth_scale(_ptr(a), _ptr(W), N, K, K, float(alpha), _ptr(s), _ptr(inv_s))
+    if normalize:
+        lib().oracle_smooth_scale_normalize(_ptr(s), _ptr(inv_s), K)
     return s, inv_s
 
 
@@ -183,6 +195,96 @@ def outlier_product(X, W, idx) -> np.ndarray:
     o = np.empty((M, N), np.float64)
     lib().oracle_outlier_product(_ptr(X), K, _ptr(W), K, M, N, _ptr(idx), int(idx.size), _ptr(o))
     return o
+
+
+# ------------------------------------------------------------------ variants
+def quant_act_per_tensor(X, inv_s: Optional[np.ndarray] = None, clip: Optional[float] = None):
+    """Per-tensor activation quantization: returns (Xq int8 [M,K], d fp32 [1]). ``clip``: a
+    static calibration value (e.g. a percentile of |X|) used instead of the tensor's absmax."""
+    X = _c(X, np.uint16)
+    inv_s = _c(inv_s, np.float32)
+    M, K = X.shape
+    Xq = np.empty((M, K), np.int8)
+    d = np.empty(1, np.float32)
+    lib().oracle_quant_act_per_tensor(_ptr(X), M, K, K, _ptr(inv_s), -1.0 if clip is None else float(clip),
+                                      _ptr(Xq), _ptr(d))
+    return Xq, d
+
+
+def norm_smooth_quant(X, norm: int, gamma, beta=None, eps: float = 1e-5, inv_s: Optional[np.ndarray] = None):
+    """LayerNorm (NORM_LAYER) or RMSNorm (NORM_RMS) with bf16 gamma/beta, smoothing and
+    per-token quantization in one pass: returns (Xq int8 [M,K], d fp32 [M], y fp32 [M,K])."""
+    X = _c(X, np.uint16)
+    gamma = _c(gamma, np.uint16)
+    beta = _c(beta, np.uint16)
+    inv_s = _c(inv_s, np.float32)
+    M, K = X.shape
+    Xq = np.empty((M, K), np.int8)
+    d = np.empty(M, np.float32)
+    y = np.empty((M, K), np.float32)
+    lib().oracle_norm_smooth_quant(_ptr(X), M, K, K, int(norm), _ptr(gamma), _ptr(beta), float(eps), _ptr(inv_s),
+                                   _ptr(Xq), _ptr(d), _ptr(y))
+    return Xq, d, y
+
+
+def mean_std_threshold(X, k: float):
+    """Returns (threshold fp32 = fp32(mean + k*std), mean fp64, std fp64) over all of X."""
+    X = _c(X, np.uint16)
+    M, K = X.shape
+    mean, sd = C.c_double(0.0), C.c_double(0.0)
+    t = lib().oracle_mean_std_threshold(_ptr(X), M, K, K, float(k), C.addressof(mean), C.addressof(sd))
+    return np.float32(t), mean.value, sd.value
+
+
+def abs_percentile(X, p: float) -> np.float32:
+    """Nearest-rank p-th percentile of |X| over all elements."""
+    X = _c(X, np.uint16)
+    M, K = X.shape
+    return np.float32(lib().oracle_abs_percentile(_ptr(X), M, K, K, float(p)))
+
+
+def quant_act_per_token_asym(X, inv_s: Optional[np.ndarray] = None):
+    """Asymmetric per-token quantization: returns (Xq int8 [M,K], d fp32 [M], z int32 [M])."""
+    X = _c(X, np.uint16)
+    inv_s = _c(inv_s, np.float32)
+    M, K = X.shape
+    Xq = np.empty((M, K), np.int8)
+    d = np.empty(M, np.float32)
+    z = np.empty(M, np.int32)
+    lib().oracle_quant_act_per_token_asym(_ptr(X), M, K, K, _ptr(inv_s), _ptr(Xq), _ptr(d), _ptr(z))
+    return Xq, d, z
+
+
+def weight_row_sums(Wq) -> np.ndarray:
+    """rs[n] = sum_k Wq[n,k] (int32)."""
+    Wq = _c(Wq, np.int8)
+    N, K = Wq.shape
+    rs = np.empty(N, np.int32)
+    lib().oracle_weight_row_sums(_ptr(Wq), N, K, _ptr(rs))
+    return rs
+
+
+def dequant_ex(acc, d, e, bias=None, x_zero=None, rs=None):
+    """Dequantization with d per token ([M]) or per tensor ([1]), e per channel or per tensor,
+    and the exact zero-point correction acc - z_m*rs_n when ``x_zero`` is given.
+    Returns (y_ref fp64 [M,N], y_bf16 uint16 [M,N])."""
+    acc = _c(acc, np.int32)
+    d = _c(d, np.float32)
+    e = _c(e, np.float32)
+    bias = _c(bias, np.uint16)
+    x_zero = _c(x_zero, np.int32)
+    rs = _c(rs, np.int32)
+    M, N = acc.shape
+    if (x_zero is None) != (rs is None):
+        raise ValueError("x_zero and rs go together")
+    y_ref = np.empty((M, N), np.float64)
+    y_bf = np.empty((M, N), np.uint16)
+    if d.size not in (1, M) or e.size not in (1, N):
+        raise ValueError("d must have 1 or M entries and e 1 or N")
+    lib().oracle_dequant_ex(_ptr(acc), M, N, _ptr(d), 1 if d.size == M else 0,
+                            _ptr(e), 1 if e.size == N else 0, _ptr(x_zero), _ptr(rs), _ptr(bias), _ptr(y_ref),
+                            _ptr(y_bf))
+    return y_ref, y_bf
 
 
 def smoothquant_linear(X, W, bias=None, alpha: float = 0.5, gran: int = PER_CHANNEL, calib=None,

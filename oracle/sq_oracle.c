@@ -16,6 +16,8 @@
  *   [BASICS]  "量化基础与INT8" (quantization fundamentals and INT8)
  *   [LLMINT8] "LLM.int8()技术解析：8位量化如何优化大语言模型计算"
  *   [SQ]      "SmoothQuant量化实战：W8A8推理部署与单节点530B模型落地"
+ *   [QAT]     "从自动驾驶芯片到大语言模型INT8量化训练实战解析" (mean + 3 std outliers)
+ *   [PREC]    "大语言模型轻量化与量化精度" (choosing quantization precision; §3.2 calibration)
  *
  * Readings of the pages that the code takes (where they are silent or differ):
  *   - quantize by multiplying with a once-per-row fp32 reciprocal r = 127/absmax
@@ -32,6 +34,27 @@
  *     than the threshold; the activation row scale is taken over the other
  *     columns only and the outlier columns get code 0; the outlier product uses
  *     the original bf16 values ([LLMINT8] §2.1, §3.1).
+ *
+ * Variants (functions after oracle_outlier_product), readings:
+ *   - per-tensor activation scale ([SQ] §3.4 forward: x_max over the whole tensor),
+ *     or a given clip value (static calibration), codes saturate by the clamp;
+ *   - normalisation s <- max(s / max_j s_j * 127, 1e-5) of [SQ] §3.3, in fp32 in
+ *     that order, inv_s = 1/s;
+ *   - fused normalisation before smoothing ([SQ] §4.2, §4.5 second detail: the
+ *     smoothing folds into the LayerNorm output): row statistics summed in fp64
+ *     and rounded once to fp32 (mean, 1/sqrt(var + eps)), then
+ *     y = ((x - mean) * rstd) * gamma + beta in fp32 (RMSNorm: y = (x * rstd) * gamma),
+ *     x' = y * inv_s, then per-token quantization as above;
+ *   - dynamic outlier threshold mu + k*sigma over all elements of X ([LLMINT8]
+ *     §3.1 pre-screening, [QAT] §2.1), mean and unbiased standard deviation in
+ *     fp64, threshold rounded once to fp32;
+ *   - percentile calibration ([PREC] §3.2): nearest-rank percentile of |X|
+ *     over all elements, rank = ceil(p/100 * n) (at least 1);
+ *   - asymmetric per-token activations ([BASICS] asymmetric quantization) over
+ *     the range [min(0, min x'), max(0, max x')] so that 0 is exact:
+ *     r = 255/range, d = range/255, z = -128 - rne(lo * r),
+ *     q = clamp(rne(x' * r) + z, -128, 127), x' ~ d * (q - z); the GEMM result is
+ *     corrected exactly in integers: acc - z_m * sum_k Wq[n,k].
  */
 #include <math.h>
 #include <stdint.h>
@@ -275,6 +298,231 @@ void oracle_outlier_product(const uint16_t *X, int64_t ldx, const uint16_t *W, i
                 t += (double)bf16_to_float(X[m * ldx + j]) * (double)bf16_to_float(W[n * ldw + j]);
             }
             o[m * N + n] = t;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ variants */
+
+/* Per-tensor activation quantization, [SQ] §3.4 SmoothQuantLinear.forward
+ * (x_max = x.abs().max(); x_scale = x_max/127; round(x/x_scale).clamp(-128,127)):
+ *   x' = X * inv_s (inv_s NULL: 1); a = clip if clip >= 0 (static calibration, e.g. a
+ *   percentile), else max over all |x'|; x_scale[0] = a/127; q = clamp(rne(x' * (127/a))). */
+void oracle_quant_act_per_tensor(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                 const float *inv_s, float clip, int8_t *Xq, float *x_scale) {
+    float a = clip;
+    if (!(clip >= 0.0f)) {
+        a = 0.0f;
+        for (int64_t m = 0; m < M; ++m)
+            for (int64_t k = 0; k < K; ++k) {
+                float x = bf16_to_float(X[m * ldx + k]);
+                float v = inv_s ? x * inv_s[k] : x;
+                if (fabsf(v) > a) a = fabsf(v);
+            }
+    }
+    x_scale[0] = a / 127.0f;
+#pragma omp parallel
+    {
+        float *v = (float *)malloc(sizeof(float) * (size_t)(K > 0 ? K : 1));
+#pragma omp for schedule(static)
+        for (int64_t m = 0; m < M; ++m) {
+            for (int64_t k = 0; k < K; ++k) {
+                float x = bf16_to_float(X[m * ldx + k]);
+                v[k] = inv_s ? x * inv_s[k] : x;
+            }
+            quantize_with_absmax(v, K, a, Xq + m * K);
+        }
+        free(v);
+    }
+}
+
+/* Normalisation of the smoothing factors, [SQ] §3.3 compute_smooth_scale:
+ *   s_j <- s_j / max_i s_i * 127 (fp32, in that order); s_j <- max(s_j, 1e-5); inv_s_j = 1/s_j. */
+void oracle_smooth_scale_normalize(float *s, float *inv_s, int64_t K) {
+    float smax = 0.0f;
+    for (int64_t j = 0; j < K; ++j)
+        if (s[j] > smax) smax = s[j];
+    for (int64_t j = 0; j < K; ++j) {
+        float t = (s[j] / smax) * 127.0f;
+        if (t < 1e-5f) t = 1e-5f;
+        s[j] = t;
+        inv_s[j] = 1.0f / t;
+    }
+}
+
+#define ORACLE_NORM_LAYER 0
+#define ORACLE_NORM_RMS 1
+
+/* Normalisation + smoothing + per-token quantization of one fused pass, [SQ] §4.2 and
+ * §4.5 second detail (the smoothing folds into the LayerNorm output). Per row m:
+ *   LayerNorm: mean = sum x / K, var = sum (x - mean)^2 / K (fp64, mean from the fp64 sum);
+ *              mean_f = fp32(mean), rstd_f = fp32(1 / sqrt(var + eps));
+ *              y = ((x - mean_f) * rstd_f) * gamma_k + beta_k            (fp32, beta NULL: 0)
+ *   RMSNorm:   ms = sum x^2 / K (fp64); rstd_f = fp32(1 / sqrt(ms + eps));
+ *              y = (x * rstd_f) * gamma_k + beta_k                       (fp32, beta NULL: 0)
+ *   x' = y * inv_s_k (inv_s NULL: 1); a = max |x'|; d_m = a/127; q = clamp(rne(x' * (127/a))).
+ * gamma, beta are bf16 [K]. */
+void oracle_norm_smooth_quant(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, int norm,
+                              const uint16_t *gamma, const uint16_t *beta, float eps,
+                              const float *inv_s, int8_t *Xq, float *x_scale, float *y_out) {
+#pragma omp parallel
+    {
+        float *v = (float *)malloc(sizeof(float) * (size_t)(K > 0 ? K : 1));
+#pragma omp for schedule(static)
+        for (int64_t m = 0; m < M; ++m) {
+            const uint16_t *xr = X + m * ldx;
+            float mean_f = 0.0f, rstd_f;
+            if (norm == ORACLE_NORM_LAYER) {
+                double sum = 0.0;
+                for (int64_t k = 0; k < K; ++k) sum += (double)bf16_to_float(xr[k]);
+                double mean = sum / (double)K;
+                double ss = 0.0;
+                for (int64_t k = 0; k < K; ++k) {
+                    double c = (double)bf16_to_float(xr[k]) - mean;
+                    ss += c * c;
+                }
+                double var = ss / (double)K;
+                mean_f = (float)mean;
+                rstd_f = (float)(1.0 / sqrt(var + (double)eps));
+            } else {
+                double ss = 0.0;
+                for (int64_t k = 0; k < K; ++k) {
+                    double x = (double)bf16_to_float(xr[k]);
+                    ss += x * x;
+                }
+                rstd_f = (float)(1.0 / sqrt(ss / (double)K + (double)eps));
+            }
+            float a = 0.0f;
+            for (int64_t k = 0; k < K; ++k) {
+                float x = bf16_to_float(xr[k]);
+                float y = (norm == ORACLE_NORM_LAYER) ? (x - mean_f) * rstd_f : x * rstd_f;
+                y = y * bf16_to_float(gamma[k]);
+                if (beta) y = y + bf16_to_float(beta[k]);
+                if (y_out) y_out[m * K + k] = y;
+                v[k] = inv_s ? y * inv_s[k] : y;
+                if (fabsf(v[k]) > a) a = fabsf(v[k]);
+            }
+            x_scale[m] = a / 127.0f;
+            quantize_with_absmax(v, K, a, Xq + m * K);
+        }
+        free(v);
+    }
+}
+
+/* Dynamic outlier threshold, [LLMINT8] §3.1 pre-screening (threshold = mu + 6 sigma from
+ * the layer's activation mean and variance) and [QAT] §2.1 (mean + 3 std of all elements,
+ * torch's unbiased std): mean and std over all M*K elements in fp64 (two passes), the
+ * threshold mean + k*std rounded once to fp32. Writes mean and std when non-NULL. */
+float oracle_mean_std_threshold(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, double k,
+                                double *mean_out, double *std_out) {
+    double n = (double)M * (double)K;
+    double sum = 0.0;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t j = 0; j < K; ++j) sum += (double)bf16_to_float(X[m * ldx + j]);
+    double mean = sum / n;
+    double ss = 0.0;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t j = 0; j < K; ++j) {
+            double c = (double)bf16_to_float(X[m * ldx + j]) - mean;
+            ss += c * c;
+        }
+    double sd = n > 1.0 ? sqrt(ss / (n - 1.0)) : 0.0;
+    if (mean_out) *mean_out = mean;
+    if (std_out) *std_out = sd;
+    return (float)(mean + k * sd);
+}
+
+static int cmp_float(const void *a, const void *b) {
+    float x = *(const float *)a, y = *(const float *)b;
+    return (x > y) - (x < y);
+}
+
+/* Percentile calibration, [PREC] §3.2 (a max calibrator with the percentile method,
+ * 99.99): the nearest-rank p-th percentile of |X| over all M*K elements: sort the absolute
+ * values ascending and take the element of 1-based rank ceil(p/100 * n), at least 1. */
+float oracle_abs_percentile(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, double p) {
+    int64_t n = M * K;
+    float *v = (float *)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t j = 0; j < K; ++j) v[m * K + j] = fabsf(bf16_to_float(X[m * ldx + j]));
+    qsort(v, (size_t)n, sizeof(float), cmp_float);
+    int64_t rank = (int64_t)ceil((p / 100.0) * (double)n);
+    if (rank < 1) rank = 1;
+    if (rank > n) rank = n;
+    float r = v[rank - 1];
+    free(v);
+    return r;
+}
+
+/* Asymmetric per-token activation quantization, [BASICS] asymmetric quantization
+ * (scale = (max - min)/255 with a zero point), on signed 8-bit codes, over the range
+ * extended to contain 0:
+ *   x' = X * inv_s; lo = min(0, min_k x'), hi = max(0, max_k x'); range = hi - lo (fp32);
+ *   r = range > 0 ? 255/range : 0; d_m = range/255; z_m = -128 - rne(lo * r);
+ *   q = clamp(rne(x' * r) + z_m, -128, 127);  x' ~ d_m * (q - z_m). */
+void oracle_quant_act_per_token_asym(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
+                                     const float *inv_s, int8_t *Xq, float *x_scale,
+                                     int32_t *x_zero) {
+#pragma omp parallel
+    {
+        float *v = (float *)malloc(sizeof(float) * (size_t)(K > 0 ? K : 1));
+#pragma omp for schedule(static)
+        for (int64_t m = 0; m < M; ++m) {
+            float lo = 0.0f, hi = 0.0f;
+            for (int64_t k = 0; k < K; ++k) {
+                float x = bf16_to_float(X[m * ldx + k]);
+                v[k] = inv_s ? x * inv_s[k] : x;
+                if (v[k] < lo) lo = v[k];
+                if (v[k] > hi) hi = v[k];
+            }
+            float range = hi - lo;
+            float r = range > 0.0f ? 255.0f / range : 0.0f;
+            int32_t z = -128 - (int32_t)nearbyintf(lo * r);
+            x_scale[m] = range / 255.0f;
+            x_zero[m] = z;
+            for (int64_t k = 0; k < K; ++k) {
+                float t = nearbyintf(v[k] * r) + (float)z;
+                if (t > 127.0f) t = 127.0f;
+                if (t < -128.0f) t = -128.0f;
+                Xq[m * K + k] = (int8_t)t;
+            }
+        }
+        free(v);
+    }
+}
+
+/* Row sums of the int8 weight, rs_n = sum_k Wq[n,k] (the zero-point correction term of an
+ * asymmetric activation: sum_k (q - z) w = sum_k q w - z * rs_n). */
+void oracle_weight_row_sums(const int8_t *Wq, int64_t N, int64_t K, int32_t *rs) {
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        int64_t t = 0;
+        for (int64_t k = 0; k < K; ++k) t += Wq[n * K + k];
+        rs[n] = (int32_t)t;
+    }
+}
+
+/* Dequantization with the variants' operands: d per token ([M]) or per tensor ([1]),
+ * e per channel ([N]) or per tensor ([1]); with x_zero (int32 [M]) and rs (int32 [N])
+ * the accumulator is first corrected exactly, a = acc - z_m * rs_n (int64):
+ *   y_ref = a * d * e + bias (fp64), y_bf16 = bf16_rne(((float)a * d) * e + bias). */
+void oracle_dequant_ex(const int32_t *acc, int64_t M, int64_t N, const float *d, int d_per_token,
+                       const float *e, int e_per_channel, const int32_t *x_zero, const int32_t *rs,
+                       const uint16_t *bias, double *y_ref, uint16_t *y_bf16) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            float dm = d_per_token ? d[m] : d[0];
+            float en = e_per_channel ? e[n] : e[0];
+            float bn = bias ? bf16_to_float(bias[n]) : 0.0f;
+            int64_t a = acc[m * N + n];
+            if (x_zero) a -= (int64_t)x_zero[m] * (int64_t)rs[n];
+            if (y_ref) y_ref[m * N + n] = (double)a * (double)dm * (double)en + (double)bn;
+            if (y_bf16) {
+                float y = ((float)a * dm) * en;
+                y = y + bn;
+                y_bf16[m * N + n] = float_to_bf16_rne(y);
+            }
         }
     }
 }

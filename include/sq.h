@@ -11,6 +11,8 @@
  *   [BASICS]  "量化基础与INT8" (quantization fundamentals and INT8)
  *   [LLMINT8] "LLM.int8()技术解析：8位量化如何优化大语言模型计算"
  *   [SQ]      "SmoothQuant量化实战：W8A8推理部署与单节点530B模型落地"
+ *   [QAT]     "从自动驾驶芯片到大语言模型INT8量化训练实战解析"
+ *   [PREC]    "大语言模型轻量化与量化精度" (choosing quantization precision)
  *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE memory owned by the caller; the library keeps no
@@ -66,10 +68,15 @@ typedef enum {
 
 typedef enum { SQ_PER_TENSOR = 0, SQ_PER_CHANNEL = 1 } sq_gran;
 
+typedef enum { SQ_NORM_LAYER = 0, SQ_NORM_RMS = 1 } sq_norm;
+
 typedef enum {
   SQ_OP_SMOOTH_QUANT_WEIGHT = 1,
-  SQ_OP_INT8_GEMM_DEQUANT = 2,
-  SQ_OP_LLMINT8 = 3
+  SQ_OP_INT8_GEMM_DEQUANT = 2, /* also sq_int8_gemm_dequant_ex */
+  SQ_OP_LLMINT8 = 3,           /* also llmint8_decomposed_linear_ex */
+  SQ_OP_QUANT_ACT_PER_TENSOR = 4,
+  SQ_OP_MEAN_STD_THRESHOLD = 5,
+  SQ_OP_ABS_PERCENTILE = 6
 } sq_op;
 
 /*
@@ -193,6 +200,129 @@ SQ_API sq_status llmint8_decomposed_linear(const void* X_bf16, const void* W_bf1
 SQ_API sq_status sq_smooth_quant_weight_noalloc(const void* W_bf16, int64_t N, int64_t K, int64_t ldw,
                                                 const float* s, sq_gran gran, int8_t* Wq, float* w_scale,
                                                 sq_stream_t stream);
+
+/* ============================================================================ variants
+ * The calls below add the variants the pages describe beside the method: a per-tensor
+ * activation scale (dynamic or calibrated), the normalisation of the smoothing factors,
+ * normalisation layers fused with smoothing and quantization, a data-dependent outlier
+ * threshold, percentile calibration and asymmetric (zero-point) activations. They follow
+ * the conventions above. */
+
+/*
+ * Per-tensor activation quantization. [SQ] §3.4 SmoothQuantLinear.forward (x_max =
+ * x.abs().max() over the whole tensor, x_scale = x_max/127, round().clamp(-128, 127)):
+ *   x'[m,k] = X[m,k] * inv_s[k]     (fp32; inv_s == NULL means 1)
+ *   a = *clip when clip != NULL (a static calibration value, e.g. from sq_act_abs_percentile;
+ *       values beyond it saturate at the clamp), else max |x'| over the tensor
+ *   x_scale[0] = a/127, Xq[m,k] = clamp(rne(x' * (127/a)), -128, 127)
+ * X: bf16 [M, K], ldx. clip: fp32 [1] device or NULL. Xq: int8 [M, K]. x_scale: fp32 [1].
+ * ws: with clip == NULL, sq_workspace_size(SQ_OP_QUANT_ACT_PER_TENSOR, M, 0, K) bytes (the
+ * running maximum); with a clip none (ws may be NULL). Two passes over X without a clip.
+ */
+SQ_API sq_status sq_quant_act_per_tensor(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, const float* inv_s,
+                                         const float* clip, int8_t* Xq, float* x_scale, void* ws, size_t ws_bytes,
+                                         sq_stream_t stream);
+
+/*
+ * Smoothing factors with the optional normalisation of [SQ] §3.3 compute_smooth_scale:
+ * normalize == 0 is sq_smooth_scale; otherwise, after s is formed,
+ *   s_j <- max( (s_j / max_i s_i) * 127, 1e-5 )   (fp32, in that order),  inv_s_j = 1/s_j.
+ * Any positive s keeps X.W^T = (X diag(s)^-1)(diag(s) W)^T, so the layer's result is the
+ * same function; only the split of the quantization difficulty moves.
+ */
+SQ_API sq_status sq_smooth_scale_ex(const float* act_amax, const void* W_bf16, int64_t N, int64_t K, int64_t ldw,
+                                    float alpha, int normalize, float* s, float* inv_s, sq_stream_t stream);
+
+/*
+ * INT8 GEMM + dequantization with the variants' activation forms:
+ *   x_gran SQ_PER_CHANNEL: x_scale is per token, fp32 [M] (as sq_int8_gemm_dequant);
+ *   x_gran SQ_PER_TENSOR : x_scale is fp32 [1] (sq_quant_act_per_tensor).
+ *   x_zero (int32 [M], per-token zero points from sq_quant_act_per_token_asym) with
+ *   w_rowsum (int32 [N], sum_k Wq[n,k] from sq_weight_row_sums): the accumulator is
+ *   corrected exactly before the dequantization, [BASICS] asymmetric quantization
+ *   (x ~ scale * (q - z), so sum_k (q - z) w = acc - z * rowsum):
+ *     acc'[m,n] = acc[m,n] - x_zero[m] * w_rowsum[n]     (64-bit integer arithmetic)
+ *     Y[m,n]    = bf16_rne( (float(acc') * x_scale[m]) * w_scale[n or 0] + bias[n] )
+ *   x_zero needs x_gran == SQ_PER_CHANNEL and a w_rowsum; x_zero == NULL is symmetric.
+ * Everything else as sq_int8_gemm_dequant (acc_out receives the uncorrected acc; ws is
+ * sized by SQ_OP_INT8_GEMM_DEQUANT).
+ */
+SQ_API sq_status sq_int8_gemm_dequant_ex(const int8_t* Xq, const int8_t* Wq, const float* x_scale, sq_gran x_gran,
+                                         const int32_t* x_zero, const float* w_scale, sq_gran w_gran,
+                                         const int32_t* w_rowsum, const void* bias_bf16, void* Y_bf16, int64_t M,
+                                         int64_t N, int64_t K, int32_t* acc_out, void* ws, size_t ws_bytes,
+                                         sq_stream_t stream);
+
+/*
+ * Normalisation layer, smoothing and per-token quantization in one pass over X: the
+ * smoothing folded into the output of the LayerNorm that precedes the linear layer
+ * ([SQ] §4.2 fuse the scaling into the previous operation's output; §4.5 second detail).
+ * Per row m, statistics summed in fp64 and rounded once to fp32:
+ *   SQ_NORM_LAYER: mean = sum_k x / K, var = sum_k (x - mean)^2 / K,
+ *                  rstd = fp32(1/sqrt(var + eps)), y = ((x - fp32(mean)) * rstd) * gamma_k + beta_k
+ *   SQ_NORM_RMS:   rstd = fp32(1/sqrt(sum_k x^2 / K + eps)),   y = (x * rstd) * gamma_k + beta_k
+ *   x' = y * inv_s_k (inv_s == NULL means 1), a_m = max_k |x'|, x_scale[m] = a_m/127,
+ *   Xq[m,k] = clamp(rne(x' * (127/a_m)), -128, 127)                  (fp32, no contraction)
+ * X: bf16 [M, K], ldx. gamma: bf16 [K]. beta: bf16 [K] or NULL (0). eps >= 0.
+ * mean_rstd: fp32 [M, 2] (fp32(mean) or 0 for RMS, rstd) or NULL. K <= 16384.
+ */
+SQ_API sq_status sq_norm_smooth_quant(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, sq_norm norm,
+                                      const void* gamma_bf16, const void* beta_bf16, float eps, const float* inv_s,
+                                      int8_t* Xq, float* x_scale, float* mean_rstd, sq_stream_t stream);
+
+/*
+ * Data-dependent outlier threshold: threshold = mean + k * std over all M*K elements of X,
+ * std the unbiased standard deviation. [LLMINT8] §3.1 pre-screening (threshold = mu + 6
+ * sigma from the layer's activation statistics); [QAT] §2.1 (mean + 3 std).
+ * mean and the sum of squared deviations are summed in fp64 (two passes over X, fixed
+ * summation order: the result is deterministic); the threshold is rounded once to fp32.
+ * threshold: fp32 [1] device. mean_std: fp64 [2] device (mean, std) or NULL.
+ * ws: sq_workspace_size(SQ_OP_MEAN_STD_THRESHOLD, M, 0, K) bytes.
+ */
+SQ_API sq_status sq_act_mean_std_threshold(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, double k,
+                                           float* threshold, double* mean_std, void* ws, size_t ws_bytes,
+                                           sq_stream_t stream);
+
+/*
+ * llmint8_decomposed_linear with the threshold read from device memory (for instance the
+ * output of sq_act_mean_std_threshold), so that a data-dependent threshold needs no host
+ * round trip. threshold: fp32 [1] device. Everything else as llmint8_decomposed_linear.
+ */
+SQ_API sq_status llmint8_decomposed_linear_ex(const void* X_bf16, const void* W_bf16, const int8_t* Wq,
+                                              const float* w_scale, const float* threshold, const void* bias_bf16,
+                                              void* Y_bf16, int64_t M, int64_t N, int64_t K, uint32_t* mask_out,
+                                              int32_t* n_outliers_out, int32_t* acc_out, void* ws, size_t ws_bytes,
+                                              sq_stream_t stream);
+
+/*
+ * Percentile calibration: the nearest-rank p-th percentile of |X| over all n = M*K
+ * elements, [PREC] §3.2 (a max calibrator with the percentile method, 99.99): the element
+ * of 1-based rank ceil(p/100 * n) (at least 1) of the ascending absolute values. Exact (a
+ * histogram of the 2^15 bf16 magnitudes and a scan). 0 <= p <= 100.
+ * out: fp32 [1] device. ws: sq_workspace_size(SQ_OP_ABS_PERCENTILE, M, 0, K) bytes.
+ */
+SQ_API sq_status sq_act_abs_percentile(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, double p, float* out,
+                                       void* ws, size_t ws_bytes, sq_stream_t stream);
+
+/*
+ * Asymmetric per-token activation quantization, [BASICS] asymmetric quantization
+ * (scale = (max - min)/255 and a zero point), on signed codes and over the row's range
+ * extended to contain 0 (so that 0 is represented exactly):
+ *   x' = X * inv_s (inv_s == NULL means 1); lo = min(0, min_k x'), hi = max(0, max_k x')
+ *   range = hi - lo, r = 255/range (0 if range == 0), x_scale[m] = range/255,
+ *   x_zero[m] = -128 - rne(lo * r), Xq[m,k] = clamp(rne(x' * r) + x_zero[m], -128, 127)
+ *   so that x' ~ x_scale[m] * (Xq - x_zero[m]).
+ * X: bf16 [M, K], ldx. Xq: int8 [M, K]. x_scale: fp32 [M]. x_zero: int32 [M].
+ */
+SQ_API sq_status sq_quant_act_per_token_asym(const void* X_bf16, int64_t M, int64_t K, int64_t ldx,
+                                             const float* inv_s, int8_t* Xq, float* x_scale, int32_t* x_zero,
+                                             sq_stream_t stream);
+
+/*
+ * Row sums of an int8 weight, rowsum[n] = sum_k Wq[n,k] (exact int32): the zero-point
+ * correction term of sq_int8_gemm_dequant_ex. Wq: int8 [N, K]. rowsum: int32 [N].
+ */
+SQ_API sq_status sq_weight_row_sums(const int8_t* Wq, int64_t N, int64_t K, int32_t* rowsum, sq_stream_t stream);
 
 /* Bytes of scratch an operation needs for the given shape (0 if none). Returns 0 for an
  * unknown op; never fails otherwise. */

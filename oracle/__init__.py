@@ -56,7 +56,7 @@ def lib():
             "oracle_outlier_product": ([p, i64, p, i64, i64, i64, p, C.c_int32, p], None),
             "oracle_quant_act_per_tensor": ([p, i64, i64, i64, p, f32, p, p], None),
             "oracle_smooth_scale_normalize": ([p, p, i64], None),
-            "oracle_norm_smooth_quant": ([p, i64, i64, i64, i32, p, p, f32, p, p, p, p], None),
+            "oracle_norm_smooth_quant": ([p, i64, i64, i64, i32, p, p, f32, p, p, p, p, p, i32], None),
             "oracle_mean_std_threshold": ([p, i64, i64, i64, C.c_double, p, p], f32),
             "oracle_abs_percentile": ([p, i64, i64, i64, C.c_double], f32),
             "oracle_quant_act_per_token_asym": ([p, i64, i64, i64, p, p, p, p], None),
@@ -211,9 +211,12 @@ def quant_act_per_tensor(X, inv_s: Optional[np.ndarray] = None, clip: Optional[f
     return Xq, d
 
 
-def norm_smooth_quant(X, norm: int, gamma, beta=None, eps: float = 1e-5, inv_s: Optional[np.ndarray] = None):
+def norm_smooth_quant(X, norm: int, gamma, beta=None, eps: float = 1e-5, inv_s: Optional[np.ndarray] = None,
+                      stats: Optional[np.ndarray] = None, with_stats: bool = False):
     """LayerNorm (NORM_LAYER) or RMSNorm (NORM_RMS) with bf16 gamma/beta, smoothing and
-    per-token quantization in one pass: returns (Xq int8 [M,K], d fp32 [M], y fp32 [M,K])."""
+    per-token quantization in one pass: returns (Xq int8 [M,K], d fp32 [M], y fp32 [M,K]),
+    plus the row statistics fp32 [M,2] (mean or 0, rstd) with ``with_stats``. ``stats``
+    supplies the statistics instead of computing them."""
     X = _c(X, np.uint16)
     gamma = _c(gamma, np.uint16)
     beta = _c(beta, np.uint16)
@@ -222,9 +225,19 @@ def norm_smooth_quant(X, norm: int, gamma, beta=None, eps: float = 1e-5, inv_s: 
     Xq = np.empty((M, K), np.int8)
     d = np.empty(M, np.float32)
     y = np.empty((M, K), np.float32)
+    given = stats is not None
+    st = np.array(stats, np.float32, copy=True).reshape(M, 2) if given else np.empty((M, 2), np.float32)
     lib().oracle_norm_smooth_quant(_ptr(X), M, K, K, int(norm), _ptr(gamma), _ptr(beta), float(eps), _ptr(inv_s),
-                                   _ptr(Xq), _ptr(d), _ptr(y))
-    return Xq, d, y
+                                   _ptr(Xq), _ptr(d), _ptr(y), _ptr(st), 1 if given else 0)
+    return (Xq, d, y, st) if with_stats else (Xq, d, y)
+
+
+def smooth_scale_normalize(s):
+    """The normalisation step alone on given factors: returns (s', inv_s') fp32 [K]."""
+    s2 = np.array(s, np.float32, copy=True)
+    inv = np.empty_like(s2)
+    lib().oracle_smooth_scale_normalize(_ptr(s2), _ptr(inv), s2.size)
+    return s2, inv
 
 
 def mean_std_threshold(X, k: float):

@@ -361,10 +361,14 @@ void oracle_smooth_scale_normalize(float *s, float *inv_s, int64_t K) {
  *   RMSNorm:   ms = sum x^2 / K (fp64); rstd_f = fp32(1 / sqrt(ms + eps));
  *              y = (x * rstd_f) * gamma_k + beta_k                       (fp32, beta NULL: 0)
  *   x' = y * inv_s_k (inv_s NULL: 1); a = max |x'|; d_m = a/127; q = clamp(rne(x' * (127/a))).
- * gamma, beta are bf16 [K]. */
+ * gamma, beta are bf16 [K]. stats [M,2] (mean_f or 0 for RMSNorm, rstd_f) receives the row
+ * statistics, or, with stats_given, supplies them: fp64 sums in another order may round
+ * to a neighbouring fp32 value, so the steps after the statistics can be checked on the
+ * statistics another implementation produced. */
 void oracle_norm_smooth_quant(const uint16_t *X, int64_t M, int64_t K, int64_t ldx, int norm,
                               const uint16_t *gamma, const uint16_t *beta, float eps,
-                              const float *inv_s, int8_t *Xq, float *x_scale, float *y_out) {
+                              const float *inv_s, int8_t *Xq, float *x_scale, float *y_out,
+                              float *stats, int stats_given) {
 #pragma omp parallel
     {
         float *v = (float *)malloc(sizeof(float) * (size_t)(K > 0 ? K : 1));
@@ -372,7 +376,10 @@ void oracle_norm_smooth_quant(const uint16_t *X, int64_t M, int64_t K, int64_t l
         for (int64_t m = 0; m < M; ++m) {
             const uint16_t *xr = X + m * ldx;
             float mean_f = 0.0f, rstd_f;
-            if (norm == ORACLE_NORM_LAYER) {
+            if (stats && stats_given) {
+                mean_f = stats[2 * m];
+                rstd_f = stats[2 * m + 1];
+            } else if (norm == ORACLE_NORM_LAYER) {
                 double sum = 0.0;
                 for (int64_t k = 0; k < K; ++k) sum += (double)bf16_to_float(xr[k]);
                 double mean = sum / (double)K;
@@ -391,6 +398,10 @@ void oracle_norm_smooth_quant(const uint16_t *X, int64_t M, int64_t K, int64_t l
                     ss += x * x;
                 }
                 rstd_f = (float)(1.0 / sqrt(ss / (double)K + (double)eps));
+            }
+            if (stats && !stats_given) {
+                stats[2 * m] = mean_f;
+                stats[2 * m + 1] = rstd_f;
             }
             float a = 0.0f;
             for (int64_t k = 0; k < K; ++k) {

@@ -92,8 +92,19 @@ def llmint8_gpu(p, threshold=None, acc=True, rows=None):
     return res
 
 
+FROB_MIN_ELEMENTS = 4096
+BF16_U = 2.0 ** -8  # unit roundoff of bf16 (8 significant bits)
+
+
 def assert_close_bf16(y_bits, y_ref, what=""):
-    """bf16 output vs the fp64 reference: max-abs <= 1e-2 max|ref|, rel-Frobenius <= 2e-3."""
+    """bf16 output vs the fp64 reference: max-abs <= 1e-2 max|ref|, rel-Frobenius <= 2e-3.
+
+    Rounding the exact result to bf16 alone gives a relative Frobenius error of about
+    1.66e-3 on large outputs, but on outputs of a few dozen elements it scatters above 2e-3
+    (the per-element bound is 2^-8 = 3.9e-3). Outputs with fewer than FROB_MIN_ELEMENTS
+    elements are therefore checked element by element against that rounding bound instead
+    of the Frobenius norm (the bit-for-bit check against the oracle's fp32 sequence, made
+    beside this one, is the strict test there)."""
     y = wl.bf16_bits_to_f32(y_bits).astype(np.float64)
     ref = np.asarray(y_ref, np.float64)
     assert np.all(np.isfinite(y)), f"{what}: non-finite output"
@@ -101,5 +112,9 @@ def assert_close_bf16(y_bits, y_ref, what=""):
     err = np.abs(y - ref)
     frob = np.linalg.norm(y - ref) / max(np.linalg.norm(ref), 1e-300)
     assert err.max() <= MAX_ABS_REL * scale + 1e-30, f"{what}: max abs err {err.max():.3e} vs {scale:.3e}"
-    assert frob <= REL_FROB, f"{what}: rel Frobenius {frob:.3e}"
+    if y.size >= FROB_MIN_ELEMENTS:
+        assert frob <= REL_FROB, f"{what}: rel Frobenius {frob:.3e}"
+    else:
+        bound = BF16_U * (1 + 2.0 ** -10) * np.abs(ref) + 1e-6 * scale
+        assert np.all(err <= bound), f"{what}: element beyond the bf16 rounding bound"
     return float(err.max() / max(scale, 1e-300)), float(frob)

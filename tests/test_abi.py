@@ -92,3 +92,50 @@ def test_llmint8_validation():
                                        None, FAKE, need - 1, None) == sq.SQ_ERR_WORKSPACE
     assert L.llmint8_decomposed_linear(FAKE, FAKE, FAKE, FAKE, C.c_float(float("nan")), None, FAKE, 16, 16, 64,
                                        None, None, None, FAKE, need, None) == sq.SQ_ERR_INVALID
+
+
+def test_variant_workspace_sizes():
+    assert sq.sq_workspace_size(sq.SQ_OP_QUANT_ACT_PER_TENSOR, 16, 0, 64) >= 4
+    assert sq.sq_workspace_size(sq.SQ_OP_MEAN_STD_THRESHOLD, 4096, 0, 8192) >= 8 * (2 * 1024 + 2)
+    assert sq.sq_workspace_size(sq.SQ_OP_MEAN_STD_THRESHOLD, 3, 0, 64) >= 8 * (2 * 3 + 2)
+    assert sq.sq_workspace_size(sq.SQ_OP_ABS_PERCENTILE, 1, 0, 16) == 8 * (1 << 15)
+
+
+def test_variant_validation():
+    L = _raw()
+    # dynamic per-tensor without workspace; clip misaligned
+    assert L.sq_quant_act_per_tensor(FAKE, 4, 64, 64, None, None, FAKE, FAKE, None, 0, None) == sq.SQ_ERR_WORKSPACE
+    assert L.sq_quant_act_per_tensor(FAKE, 4, 64, 64, None, FAKE + 2, FAKE, FAKE, None, 0, None) == sq.SQ_ERR_ALIGN
+    # asymmetric GEMM needs per-token scales and row sums
+    assert L.sq_int8_gemm_dequant_ex(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 1, FAKE, None, FAKE, 16, 16, 64, None, None, 0,
+                                     None) == sq.SQ_ERR_INVALID
+    assert L.sq_int8_gemm_dequant_ex(FAKE, FAKE, FAKE, 1, FAKE, FAKE, 1, None, None, FAKE, 16, 16, 64, None, None, 0,
+                                     None) == sq.SQ_ERR_INVALID
+    assert L.sq_int8_gemm_dequant_ex(FAKE, FAKE, FAKE, 5, None, FAKE, 1, None, None, FAKE, 16, 16, 64, None, None, 0,
+                                     None) == sq.SQ_ERR_INVALID
+    # fused norm: K above the register-resident limit, bad norm, negative eps, no gamma
+    assert L.sq_norm_smooth_quant(FAKE, 4, 16400, 16400, 0, FAKE, None, C.c_float(1e-5), None, FAKE, FAKE, None,
+                                  None) == sq.SQ_ERR_INVALID
+    assert L.sq_norm_smooth_quant(FAKE, 4, 64, 64, 2, FAKE, None, C.c_float(1e-5), None, FAKE, FAKE, None,
+                                  None) == sq.SQ_ERR_INVALID
+    assert L.sq_norm_smooth_quant(FAKE, 4, 64, 64, 0, FAKE, None, C.c_float(-1.0), None, FAKE, FAKE, None,
+                                  None) == sq.SQ_ERR_INVALID
+    assert L.sq_norm_smooth_quant(FAKE, 4, 64, 64, 1, None, None, C.c_float(1e-5), None, FAKE, FAKE, None,
+                                  None) == sq.SQ_ERR_INVALID
+    # threshold and percentile: workspace, NaN k, p out of range
+    need = sq.sq_workspace_size(sq.SQ_OP_MEAN_STD_THRESHOLD, 4, 0, 64)
+    assert L.sq_act_mean_std_threshold(FAKE, 4, 64, 64, C.c_double(6.0), FAKE, None, FAKE, need - 8, None) \
+        == sq.SQ_ERR_WORKSPACE
+    assert L.sq_act_mean_std_threshold(FAKE, 4, 64, 64, C.c_double(float("nan")), FAKE, None, FAKE, need, None) \
+        == sq.SQ_ERR_INVALID
+    pneed = sq.sq_workspace_size(sq.SQ_OP_ABS_PERCENTILE, 4, 0, 64)
+    assert L.sq_act_abs_percentile(FAKE, 4, 64, 64, C.c_double(100.5), FAKE, FAKE, pneed, None) == sq.SQ_ERR_INVALID
+    assert L.sq_act_abs_percentile(FAKE, 4, 64, 64, C.c_double(50.0), FAKE, FAKE, pneed - 1, None) \
+        == sq.SQ_ERR_WORKSPACE
+    # asymmetric quantization and row sums: null outputs
+    assert L.sq_quant_act_per_token_asym(FAKE, 4, 64, 64, None, FAKE, FAKE, None, None) == sq.SQ_ERR_INVALID
+    assert L.sq_weight_row_sums(FAKE, 4, 64, None, None) == sq.SQ_ERR_INVALID
+    # LLM.int8 with a device threshold: NULL threshold
+    lneed = sq.sq_workspace_size(sq.SQ_OP_LLMINT8, 16, 16, 64)
+    assert L.llmint8_decomposed_linear_ex(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 16, 16, 64, None, None, None,
+                                          FAKE, lneed, None) == sq.SQ_ERR_INVALID

@@ -302,3 +302,20 @@ def test_variant_pins_catch_planted_mistakes():
     xc = _bits(np.full((1, 32), 2.0, np.float32))
     _, _, y_rms = oracle.norm_smooth_quant(xc, oracle.NORM_RMS, _bits(np.ones(32, np.float32)), None, 0.0)
     assert not np.allclose(y_rms, 0.0)
+
+
+def test_norm_statistics_round_trip():
+    """Statistics returned by the oracle and fed back reproduce its result; other statistics
+    change it (the override is really used)."""
+    rng = np.random.default_rng(16)
+    x = _bits(rng.normal(0.5, 2.0, (6, 128)).astype(np.float32))
+    g = _bits(rng.uniform(0.5, 1.5, 128).astype(np.float32))
+    q, d, y, st = oracle.norm_smooth_quant(x, oracle.NORM_LAYER, g, None, 1e-5, with_stats=True)
+    X = _f32(x).astype(np.float64)
+    assert np.all(st[:, 0] == X.mean(axis=1).astype(np.float32))
+    q2, d2, y2 = oracle.norm_smooth_quant(x, oracle.NORM_LAYER, g, None, 1e-5, stats=st)
+    assert np.array_equal(q, q2) and np.array_equal(d, d2) and np.array_equal(y, y2)
+    st3 = st.copy()
+    st3[:, 1] *= np.float32(2.0)
+    _, _, y3 = oracle.norm_smooth_quant(x, oracle.NORM_LAYER, g, None, 1e-5, stats=st3)
+    assert np.array_equal(y3, 2.0 * y)

@@ -5,6 +5,7 @@
 #include "sq_internal.h"
 
 #include <atomic>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -196,11 +197,21 @@ sq_status sq_quant_act_per_token(const void* X_bf16, int64_t M, int64_t K, int64
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
 }
 
-sq_status sq_int8_gemm_dequant(const int8_t* Xq, const int8_t* Wq, const float* x_scale, const float* w_scale,
-                               sq_gran w_gran, const void* bias_bf16, void* Y_bf16, int64_t M, int64_t N, int64_t K,
-                               int32_t* acc_out, void* ws, size_t ws_bytes, sq_stream_t stream) {
-  const char* fn = "sq_int8_gemm_dequant";
+}  // extern "C"
+
+namespace {
+
+sq_status gemm_impl(const char* fn, const int8_t* Xq, const int8_t* Wq, const float* x_scale, sq_gran x_gran,
+                    const int32_t* x_zero, const float* w_scale, sq_gran w_gran, const int32_t* w_rowsum,
+                    const void* bias_bf16, void* Y_bf16, int64_t M, int64_t N, int64_t K, int32_t* acc_out, void* ws,
+                    size_t ws_bytes, sq_stream_t stream) {
   sq_status st;
+  if (x_gran != SQ_PER_TENSOR && x_gran != SQ_PER_CHANNEL) return fail(SQ_ERR_INVALID, "%s: bad x granularity", fn);
+  if (x_zero != nullptr && (x_gran != SQ_PER_CHANNEL || w_rowsum == nullptr))
+    return fail(SQ_ERR_INVALID, "%s: x_zero needs per-token x_scale and w_rowsum", fn);
+  if ((x_zero != nullptr && (reinterpret_cast<uintptr_t>(x_zero) & 3u)) ||
+      (w_rowsum != nullptr && (reinterpret_cast<uintptr_t>(w_rowsum) & 3u)))
+    return fail(SQ_ERR_ALIGN, "%s: x_zero / w_rowsum not 4-byte aligned", fn);
   if ((st = check_rows(fn, "Xq", Xq, M, K, K)) != SQ_OK) return st;
   if ((st = check_rows(fn, "Wq", Wq, N, K, K)) != SQ_OK) return st;
   if (x_scale == nullptr || w_scale == nullptr) return fail(SQ_ERR_INVALID, "%s: scale pointer is NULL", fn);
@@ -219,6 +230,9 @@ sq_status sq_int8_gemm_dequant(const int8_t* Xq, const int8_t* Wq, const float* 
   a.Xq = Xq;
   a.Wq = Wq;
   a.x_scale = x_scale;
+  a.x_per_token = (x_gran == SQ_PER_CHANNEL);
+  a.x_zero = x_zero;
+  a.w_rowsum = w_rowsum;
   a.w_scale = w_scale;
   a.w_per_channel = (w_gran == SQ_PER_CHANNEL);
   a.bias = static_cast<const uint16_t*>(bias_bf16);
@@ -240,11 +254,10 @@ sq_status sq_int8_gemm_dequant(const int8_t* Xq, const int8_t* Wq, const float* 
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, why);
 }
 
-sq_status llmint8_decomposed_linear(const void* X_bf16, const void* W_bf16, const int8_t* Wq, const float* w_scale,
-                                    float threshold, const void* bias_bf16, void* Y_bf16, int64_t M, int64_t N,
-                                    int64_t K, uint32_t* mask_out, int32_t* n_outliers_out, int32_t* acc_out,
-                                    void* ws, size_t ws_bytes, sq_stream_t stream) {
-  const char* fn = "llmint8_decomposed_linear";
+sq_status llm_impl(const char* fn, const void* X_bf16, const void* W_bf16, const int8_t* Wq, const float* w_scale,
+                   float threshold, const float* threshold_dev, const void* bias_bf16, void* Y_bf16, int64_t M,
+                   int64_t N, int64_t K, uint32_t* mask_out, int32_t* n_outliers_out, int32_t* acc_out, void* ws,
+                   size_t ws_bytes, sq_stream_t stream) {
   sq_status st;
   if ((st = check_rows(fn, "X", X_bf16, M, K, K)) != SQ_OK) return st;
   if ((st = check_rows(fn, "W", W_bf16, N, K, K)) != SQ_OK) return st;
@@ -259,7 +272,9 @@ sq_status llmint8_decomposed_linear(const void* X_bf16, const void* W_bf16, cons
     return fail(SQ_ERR_ALIGN, "%s: n_outliers_out not 4-byte aligned", fn);
   if (N % 8 != 0) return fail(SQ_ERR_INVALID, "%s: N=%lld must be a multiple of 8", fn, static_cast<long long>(N));
   if (!tiles_fit(M, N)) return fail(SQ_ERR_INVALID, "%s: M x N too large", fn);
-  if (threshold != threshold) return fail(SQ_ERR_INVALID, "%s: threshold is NaN", fn);
+  if (threshold_dev == nullptr && threshold != threshold) return fail(SQ_ERR_INVALID, "%s: threshold is NaN", fn);
+  if (threshold_dev != nullptr && (reinterpret_cast<uintptr_t>(threshold_dev) & 3u))
+    return fail(SQ_ERR_ALIGN, "%s: threshold not 4-byte aligned", fn);
   const LlmLayout L = llm_layout(M, N, K);
   if (ws == nullptr || ws_bytes < L.total)
     return fail(SQ_ERR_WORKSPACE, "%s: needs %zu workspace bytes, got %zu", fn, L.total,
@@ -281,7 +296,8 @@ sq_status llmint8_decomposed_linear(const void* X_bf16, const void* W_bf16, cons
 
   cudaError_t e = sq::launch_col_absmax(X, M, K, K, amax, false, cs);
   if (e == cudaSuccess)
-    e = sq::launch_outlier_mask(amax, K, threshold, mask, prefix, idx, count, mask_out, n_outliers_out, cs);
+    e = sq::launch_outlier_mask(amax, K, threshold, threshold_dev, mask, prefix, idx, count, mask_out,
+                                n_outliers_out, cs);
   if (e == cudaSuccess) {
     sq::OutlierView ov;
     ov.mask = mask;
@@ -314,6 +330,166 @@ sq_status llmint8_decomposed_linear(const void* X_bf16, const void* W_bf16, cons
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, why);
 }
 
+}  // namespace
+
+extern "C" {
+
+sq_status sq_int8_gemm_dequant(const int8_t* Xq, const int8_t* Wq, const float* x_scale, const float* w_scale,
+                               sq_gran w_gran, const void* bias_bf16, void* Y_bf16, int64_t M, int64_t N, int64_t K,
+                               int32_t* acc_out, void* ws, size_t ws_bytes, sq_stream_t stream) {
+  return gemm_impl("sq_int8_gemm_dequant", Xq, Wq, x_scale, SQ_PER_CHANNEL, nullptr, w_scale, w_gran, nullptr,
+                   bias_bf16, Y_bf16, M, N, K, acc_out, ws, ws_bytes, stream);
+}
+
+sq_status sq_int8_gemm_dequant_ex(const int8_t* Xq, const int8_t* Wq, const float* x_scale, sq_gran x_gran,
+                                  const int32_t* x_zero, const float* w_scale, sq_gran w_gran, const int32_t* w_rowsum,
+                                  const void* bias_bf16, void* Y_bf16, int64_t M, int64_t N, int64_t K,
+                                  int32_t* acc_out, void* ws, size_t ws_bytes, sq_stream_t stream) {
+  return gemm_impl("sq_int8_gemm_dequant_ex", Xq, Wq, x_scale, x_gran, x_zero, w_scale, w_gran, w_rowsum, bias_bf16,
+                   Y_bf16, M, N, K, acc_out, ws, ws_bytes, stream);
+}
+
+sq_status llmint8_decomposed_linear(const void* X_bf16, const void* W_bf16, const int8_t* Wq, const float* w_scale,
+                                    float threshold, const void* bias_bf16, void* Y_bf16, int64_t M, int64_t N,
+                                    int64_t K, uint32_t* mask_out, int32_t* n_outliers_out, int32_t* acc_out,
+                                    void* ws, size_t ws_bytes, sq_stream_t stream) {
+  return llm_impl("llmint8_decomposed_linear", X_bf16, W_bf16, Wq, w_scale, threshold, nullptr, bias_bf16, Y_bf16, M,
+                  N, K, mask_out, n_outliers_out, acc_out, ws, ws_bytes, stream);
+}
+
+sq_status llmint8_decomposed_linear_ex(const void* X_bf16, const void* W_bf16, const int8_t* Wq,
+                                       const float* w_scale, const float* threshold, const void* bias_bf16,
+                                       void* Y_bf16, int64_t M, int64_t N, int64_t K, uint32_t* mask_out,
+                                       int32_t* n_outliers_out, int32_t* acc_out, void* ws, size_t ws_bytes,
+                                       sq_stream_t stream) {
+  if (threshold == nullptr) return fail(SQ_ERR_INVALID, "llmint8_decomposed_linear_ex: threshold is NULL");
+  return llm_impl("llmint8_decomposed_linear_ex", X_bf16, W_bf16, Wq, w_scale, 0.0f, threshold, bias_bf16, Y_bf16,
+                  M, N, K, mask_out, n_outliers_out, acc_out, ws, ws_bytes, stream);
+}
+
+sq_status sq_quant_act_per_tensor(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, const float* inv_s,
+                                  const float* clip, int8_t* Xq, float* x_scale, void* ws, size_t ws_bytes,
+                                  sq_stream_t stream) {
+  const char* fn = "sq_quant_act_per_tensor";
+  sq_status st = check_rows(fn, "X", X_bf16, M, K, ldx);
+  if (st != SQ_OK) return st;
+  if ((st = check_vec(fn, "inv_s", inv_s, false)) != SQ_OK) return st;
+  if ((st = check_vec(fn, "Xq", Xq, true)) != SQ_OK) return st;
+  if (x_scale == nullptr) return fail(SQ_ERR_INVALID, "%s: x_scale is NULL", fn);
+  if (clip != nullptr && (reinterpret_cast<uintptr_t>(clip) & 3u))
+    return fail(SQ_ERR_ALIGN, "%s: clip not 4-byte aligned", fn);
+  if (clip == nullptr) {
+    const size_t need = sq_workspace_size(SQ_OP_QUANT_ACT_PER_TENSOR, M, 0, K);
+    if (ws == nullptr || ws_bytes < need)
+      return fail(SQ_ERR_WORKSPACE, "%s: needs %zu workspace bytes, got %zu", fn, need,
+                  ws == nullptr ? size_t(0) : ws_bytes);
+    if ((reinterpret_cast<uintptr_t>(ws) & 3u) != 0) return fail(SQ_ERR_ALIGN, "%s: ws not 4-byte aligned", fn);
+  }
+  cudaError_t e = sq::launch_quant_tensor(static_cast<const uint16_t*>(X_bf16), M, K, ldx, inv_s,
+                                          static_cast<unsigned int*>(ws), Xq, x_scale,
+                                          reinterpret_cast<cudaStream_t>(stream), clip);
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+
+sq_status sq_smooth_scale_ex(const float* act_amax, const void* W_bf16, int64_t N, int64_t K, int64_t ldw,
+                             float alpha, int normalize, float* s, float* inv_s, sq_stream_t stream) {
+  sq_status st = sq_smooth_scale(act_amax, W_bf16, N, K, ldw, alpha, s, inv_s, stream);
+  if (st != SQ_OK || !normalize) return st;
+  cudaError_t e = sq::launch_normalize_scale(s, inv_s, K, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, "sq_smooth_scale_ex");
+}
+
+sq_status sq_norm_smooth_quant(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, sq_norm norm,
+                               const void* gamma_bf16, const void* beta_bf16, float eps, const float* inv_s,
+                               int8_t* Xq, float* x_scale, float* mean_rstd, sq_stream_t stream) {
+  const char* fn = "sq_norm_smooth_quant";
+  sq_status st = check_rows(fn, "X", X_bf16, M, K, ldx);
+  if (st != SQ_OK) return st;
+  if (K > 16384) return fail(SQ_ERR_INVALID, "%s: K=%lld above 16384", fn, static_cast<long long>(K));
+  if (norm != SQ_NORM_LAYER && norm != SQ_NORM_RMS) return fail(SQ_ERR_INVALID, "%s: bad norm", fn);
+  if (!(eps >= 0.0f) || eps == INFINITY) return fail(SQ_ERR_INVALID, "%s: eps must be finite and >= 0", fn);
+  if ((st = check_vec(fn, "gamma", gamma_bf16, true)) != SQ_OK) return st;
+  if ((st = check_vec(fn, "beta", beta_bf16, false)) != SQ_OK) return st;
+  if ((st = check_vec(fn, "inv_s", inv_s, false)) != SQ_OK) return st;
+  if ((st = check_vec(fn, "Xq", Xq, true)) != SQ_OK) return st;
+  if (x_scale == nullptr) return fail(SQ_ERR_INVALID, "%s: x_scale is NULL", fn);
+  if (mean_rstd != nullptr && (reinterpret_cast<uintptr_t>(mean_rstd) & 7u))
+    return fail(SQ_ERR_ALIGN, "%s: mean_rstd not 8-byte aligned", fn);
+  cudaError_t e = sq::launch_norm_quant(static_cast<const uint16_t*>(X_bf16), M, K, ldx, static_cast<int>(norm),
+                                        static_cast<const uint16_t*>(gamma_bf16),
+                                        static_cast<const uint16_t*>(beta_bf16), eps, inv_s, Xq, x_scale, mean_rstd,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+
+sq_status sq_act_mean_std_threshold(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, double k, float* threshold,
+                                    double* mean_std, void* ws, size_t ws_bytes, sq_stream_t stream) {
+  const char* fn = "sq_act_mean_std_threshold";
+  sq_status st = check_rows(fn, "X", X_bf16, M, K, ldx);
+  if (st != SQ_OK) return st;
+  if (threshold == nullptr) return fail(SQ_ERR_INVALID, "%s: threshold is NULL", fn);
+  if (reinterpret_cast<uintptr_t>(threshold) & 3u) return fail(SQ_ERR_ALIGN, "%s: threshold not aligned", fn);
+  if (mean_std != nullptr && (reinterpret_cast<uintptr_t>(mean_std) & 7u))
+    return fail(SQ_ERR_ALIGN, "%s: mean_std not 8-byte aligned", fn);
+  if (k != k) return fail(SQ_ERR_INVALID, "%s: k is NaN", fn);
+  const size_t need = sq_workspace_size(SQ_OP_MEAN_STD_THRESHOLD, M, 0, K);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(SQ_ERR_WORKSPACE, "%s: needs %zu workspace bytes, got %zu", fn, need,
+                ws == nullptr ? size_t(0) : ws_bytes);
+  if (reinterpret_cast<uintptr_t>(ws) & 7u) return fail(SQ_ERR_ALIGN, "%s: ws not 8-byte aligned", fn);
+  cudaError_t e = sq::launch_mean_std_threshold(static_cast<const uint16_t*>(X_bf16), M, K, ldx, k, threshold,
+                                                mean_std, ws, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+
+sq_status sq_act_abs_percentile(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, double p, float* out,
+                                void* ws, size_t ws_bytes, sq_stream_t stream) {
+  const char* fn = "sq_act_abs_percentile";
+  sq_status st = check_rows(fn, "X", X_bf16, M, K, ldx);
+  if (st != SQ_OK) return st;
+  if (out == nullptr) return fail(SQ_ERR_INVALID, "%s: out is NULL", fn);
+  if (reinterpret_cast<uintptr_t>(out) & 3u) return fail(SQ_ERR_ALIGN, "%s: out not 4-byte aligned", fn);
+  if (!(p >= 0.0 && p <= 100.0)) return fail(SQ_ERR_INVALID, "%s: p=%g outside [0, 100]", fn, p);
+  const size_t need = sq_workspace_size(SQ_OP_ABS_PERCENTILE, M, 0, K);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(SQ_ERR_WORKSPACE, "%s: needs %zu workspace bytes, got %zu", fn, need,
+                ws == nullptr ? size_t(0) : ws_bytes);
+  if (reinterpret_cast<uintptr_t>(ws) & 7u) return fail(SQ_ERR_ALIGN, "%s: ws not 8-byte aligned", fn);
+  // 1-based nearest rank, computed on the host in fp64 exactly as written
+  const int64_t n = M * K;
+  int64_t rank = static_cast<int64_t>(std::ceil((p / 100.0) * static_cast<double>(n)));
+  if (rank < 1) rank = 1;
+  if (rank > n) rank = n;
+  cudaError_t e = sq::launch_abs_percentile(static_cast<const uint16_t*>(X_bf16), M, K, ldx,
+                                            static_cast<uint64_t>(rank), out, ws,
+                                            reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+
+sq_status sq_quant_act_per_token_asym(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, const float* inv_s,
+                                      int8_t* Xq, float* x_scale, int32_t* x_zero, sq_stream_t stream) {
+  const char* fn = "sq_quant_act_per_token_asym";
+  sq_status st = check_rows(fn, "X", X_bf16, M, K, ldx);
+  if (st != SQ_OK) return st;
+  if ((st = check_vec(fn, "inv_s", inv_s, false)) != SQ_OK) return st;
+  if ((st = check_vec(fn, "Xq", Xq, true)) != SQ_OK) return st;
+  if (x_scale == nullptr || x_zero == nullptr) return fail(SQ_ERR_INVALID, "%s: x_scale / x_zero is NULL", fn);
+  if ((reinterpret_cast<uintptr_t>(x_zero) & 3u)) return fail(SQ_ERR_ALIGN, "%s: x_zero not 4-byte aligned", fn);
+  cudaError_t e = sq::launch_quant_rows_asym(static_cast<const uint16_t*>(X_bf16), M, K, ldx, inv_s, Xq, x_scale,
+                                             x_zero, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+
+sq_status sq_weight_row_sums(const int8_t* Wq, int64_t N, int64_t K, int32_t* rowsum, sq_stream_t stream) {
+  const char* fn = "sq_weight_row_sums";
+  sq_status st = check_rows(fn, "Wq", Wq, N, K, K);
+  if (st != SQ_OK) return st;
+  if (rowsum == nullptr) return fail(SQ_ERR_INVALID, "%s: rowsum is NULL", fn);
+  if (reinterpret_cast<uintptr_t>(rowsum) & 3u) return fail(SQ_ERR_ALIGN, "%s: rowsum not 4-byte aligned", fn);
+  cudaError_t e = sq::launch_row_sums(Wq, N, K, rowsum, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+
 size_t sq_workspace_size(int op, int64_t M, int64_t N, int64_t K) {
   switch (op) {
     case SQ_OP_SMOOTH_QUANT_WEIGHT:
@@ -322,6 +498,12 @@ size_t sq_workspace_size(int op, int64_t M, int64_t N, int64_t K) {
       return sq::gemm_workspace_bytes(M, N, K, false);
     case SQ_OP_LLMINT8:
       return (M < 1 || N < 1 || K < 1) ? 0 : llm_layout(M, N, K).total;
+    case SQ_OP_QUANT_ACT_PER_TENSOR:
+      return kAlign;
+    case SQ_OP_MEAN_STD_THRESHOLD:
+      return M < 1 ? 0 : sq::mean_std_workspace_bytes(M);
+    case SQ_OP_ABS_PERCENTILE:
+      return sq::abs_percentile_workspace_bytes();
     default:
       return 0;
   }

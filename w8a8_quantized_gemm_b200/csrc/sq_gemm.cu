@@ -62,6 +62,9 @@ struct Cfg {
 
 struct Params {
   const float* x_scale;
+  int x_per_token;           // x_scale has M entries (else 1)
+  const int32_t* x_zero;     // asymmetric activations: per-token zero points [M], or nullptr
+  const int32_t* w_rowsum;   // sum_k Wq[n,k] [N] (with x_zero)
   const float* w_scale;
   int w_per_channel;
   const uint16_t* bias;
@@ -146,22 +149,34 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 struct ColConsts {
   float4 e;
   uint2 b;
+  int4 z;  // asymmetric activations: the column's integer factor of the zero-point correction
 };
 
-template <bool SWAP>
+template <bool SWAP, bool ASYM>
 __device__ __forceinline__ ColConsts load_col_consts(const Params& p, int64_t n_half0, int lane, int chunks) {
   ColConsts cc;
   const int c = lane >> 3;
   const int64_t n = n_half0 + c * 32 + (lane & 7) * 4;
   const bool ok = c < chunks && n < p.cols;
+  cc.z = make_int4(0, 0, 0, 0);
   if constexpr (SWAP) {
-    // x_scale has no alignment contract and M need not be a multiple of 4: scalar loads
+    // x_scale / x_zero have no alignment contract and M need not be a multiple of 4: scalar loads
     float v[4];
+    int zz[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = (ok && n + i < p.cols) ? __ldg(p.x_scale + n + i) : 0.0f;
+    for (int i = 0; i < 4; ++i) {
+      const bool in = ok && n + i < p.cols;
+      v[i] = in ? __ldg(p.x_scale + (p.x_per_token ? n + i : 0)) : 0.0f;
+      zz[i] = (ASYM && in) ? __ldg(p.x_zero + n + i) : 0;
+    }
     cc.e = make_float4(v[0], v[1], v[2], v[3]);
     cc.b = make_uint2(0u, 0u);
+    if constexpr (ASYM) cc.z = make_int4(zz[0], zz[1], zz[2], zz[3]);
   } else {
+    if constexpr (ASYM) {
+      if (ok) cc.z = make_int4(__ldg(p.w_rowsum + n), __ldg(p.w_rowsum + n + 1), __ldg(p.w_rowsum + n + 2),
+                               __ldg(p.w_rowsum + n + 3));
+    }
     if (p.w_per_channel) {
       cc.e = ok ? __ldg(reinterpret_cast<const float4*>(p.w_scale + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
     } else {
@@ -175,18 +190,34 @@ __device__ __forceinline__ ColConsts load_col_consts(const Params& p, int64_t n_
 
 // y[j] = (float(acc[j]) * d_m) * e_n for the 32 columns of chunk c: d_m is the row
 // constant and e_n comes from the lanes' column constants, or, with swapped operands,
-// d_m comes from the column constants and e_n is the row constant.
-template <bool SWAP>
-__device__ __forceinline__ void dequant32(const uint32_t (&acc)[32], float row_scale, const ColConsts& cc, int c,
-                                          float (&y)[32]) {
+// d_m comes from the column constants and e_n is the row constant. With asymmetric
+// activations acc is first corrected in 64-bit integers, acc - z_m * rowsum_n, the row's
+// integer factor times the column's (z_m and rowsum_n, or rowsum_n and z_m if swapped).
+template <bool SWAP, bool ASYM>
+__device__ __forceinline__ void dequant32(const uint32_t (&acc)[32], float row_scale, int row_int,
+                                          const ColConsts& cc, int c, float (&y)[32]) {
 #pragma unroll
   for (int j = 0; j < 32; j += 4) {
     const int src = c * 8 + j / 4;
     const float e[4] = {__shfl_sync(0xffffffffu, cc.e.x, src), __shfl_sync(0xffffffffu, cc.e.y, src),
                         __shfl_sync(0xffffffffu, cc.e.z, src), __shfl_sync(0xffffffffu, cc.e.w, src)};
+    int zc[4] = {0, 0, 0, 0};
+    if constexpr (ASYM) {
+      zc[0] = __shfl_sync(0xffffffffu, cc.z.x, src);
+      zc[1] = __shfl_sync(0xffffffffu, cc.z.y, src);
+      zc[2] = __shfl_sync(0xffffffffu, cc.z.z, src);
+      zc[3] = __shfl_sync(0xffffffffu, cc.z.w, src);
+    }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float a = static_cast<float>(static_cast<int32_t>(acc[j + u]));
+      float a;
+      if constexpr (ASYM) {
+        const long long t = static_cast<long long>(static_cast<int32_t>(acc[j + u])) -
+                            static_cast<long long>(row_int) * static_cast<long long>(zc[u]);
+        a = __ll2float_rn(t);
+      } else {
+        a = static_cast<float>(static_cast<int32_t>(acc[j + u]));
+      }
       y[j + u] = SWAP ? __fmul_rn(__fmul_rn(a, e[u]), row_scale) : __fmul_rn(__fmul_rn(a, row_scale), e[u]);
     }
   }
@@ -272,7 +303,7 @@ __device__ __forceinline__ void store_box(const uint32_t (&v)[16], uint8_t* stag
   ebuf ^= 1;
 }
 
-template <int BN, bool OUTLIERS, int ACC_BUFS, bool SWAP>
+template <int BN, bool OUTLIERS, int ACC_BUFS, bool SWAP, bool ASYM>
 __global__ void __launch_bounds__(kThreads, 1)
 w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmXo, const __grid_constant__ CUtensorMap tmWo,
@@ -446,7 +477,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     // to the MMA warp before the stores; each 32x32 bf16 box then goes through this warp's
     // staging buffer in shared memory to a TMA store.
     constexpr int kChunks = BN / 64;  // 32-column chunks per warp
-    static_assert(!(SWAP && OUTLIERS), "swapped operands carry no outlier product");
+    static_assert(!(SWAP && OUTLIERS) && !(ASYM && OUTLIERS), "no outlier product with these forms");
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
@@ -467,15 +498,20 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const int64_t n_half0 = static_cast<int64_t>(tile_mn / p.num_m_tiles) * BN + half * (BN / 2);
       const bool r_ok = r < p.rows;
       float row_scale = 0.0f, row_bias = 0.0f;
+      int row_int = 0;
       if constexpr (SWAP) {
         if (r_ok) {
           row_scale = __ldg(p.w_scale + (p.w_per_channel ? r : 0));
           if (p.bias != nullptr) row_bias = __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + r)) << 16);
+          if constexpr (ASYM) row_int = __ldg(p.w_rowsum + r);
         }
       } else {
-        row_scale = r_ok ? __ldg(p.x_scale + r) : 0.0f;
+        if (r_ok) {
+          row_scale = __ldg(p.x_scale + (p.x_per_token ? r : 0));
+          if constexpr (ASYM) row_int = __ldg(p.x_zero + r);
+        }
       }
-      const ColConsts cc = load_col_consts<SWAP>(p, n_half0, lane, kChunks);
+      const ColConsts cc = load_col_consts<SWAP, ASYM>(p, n_half0, lane, kChunks);
       const bool has_bias = p.bias != nullptr;
       // lane 0 waits and the warp follows its verdict, so the warp stays converged
       int ok = 0;
@@ -500,7 +536,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             tmem_wait_ld();
             const int nvalid = (p.cols - n0) < 32 ? static_cast<int>(p.cols - n0) : 32;
             float y[32];
-            dequant32<SWAP>(acc, row_scale, cc, c, y);
+            dequant32<SWAP, ASYM>(acc, row_scale, row_int, cc, c, y);
             if (p.acc_out != nullptr && r_ok) store_acc32<SWAP>(p, acc, r, n0, nvalid);
             if constexpr (OUTLIERS) {
               if (kb_o > 0) {
@@ -585,7 +621,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
               }
             }
             float y[32];
-            dequant32<SWAP>(acc, row_scale, cc, c, y);
+            dequant32<SWAP, ASYM>(acc, row_scale, row_int, cc, c, y);
             if (p.acc_out != nullptr && r_ok) store_acc32<SWAP>(p, acc, r, n0, nvalid);
             uint32_t packed[16];
             bias_pack32<SWAP>(y, has_bias, cc, c, row_bias, packed);
@@ -698,7 +734,7 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool outliers) {
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
-template <int BN, bool OUTLIERS, int ACC_BUFS, bool SWAP>
+template <int BN, bool OUTLIERS, int ACC_BUFS, bool SWAP, bool ASYM = false>
 cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const char** why) {
   using C = Cfg<BN, OUTLIERS, ACC_BUFS>;
   CUtensorMap tmA{}, tmB{}, tmXo{}, tmWo{}, tmY{};
@@ -734,7 +770,7 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   cudaGetDevice(&dev);
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_done.load() & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS, SWAP>,
+    cudaError_t e = cudaFuncSetAttribute(w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS, SWAP, ASYM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) {
       *why = "cudaFuncSetAttribute(MaxDynamicSharedMemorySize) failed";
@@ -744,6 +780,9 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   }
   Params p{};
   p.x_scale = a.x_scale;
+  p.x_per_token = a.x_per_token ? 1 : 0;
+  p.x_zero = a.x_zero;
+  p.w_rowsum = a.w_rowsum;
   p.w_scale = a.w_scale;
   p.w_per_channel = a.w_per_channel ? 1 : 0;
   p.bias = a.bias;
@@ -774,7 +813,7 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   // short, latency-bound launches (swapped or K-split plans) overlap their set-up with
   // the previous kernel's tail
   const bool programmatic = SWAP || pl.tail_tiles > 0;
-  return launch_kernel(w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS, SWAP>, dim3(grid), dim3(kThreads), C::kSmemBytes,
+  return launch_kernel(w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS, SWAP, ASYM>, dim3(grid), dim3(kThreads), C::kSmemBytes,
                        stream, programmatic, tmA, tmB, tmXo, tmWo, tmY, p);
 }
 
@@ -795,6 +834,12 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream, const char** why
     if (pl.bn == 256) return run<256, true, 1, false>(a, pl, stream, why);
     if (pl.bn == 128) return run<128, true, 2, false>(a, pl, stream, why);
     return run<64, true, 2, false>(a, pl, stream, why);
+  }
+  if (a.x_zero != nullptr) {
+    if (pl.swap) return run<64, false, 2, true, true>(a, pl, stream, why);
+    if (pl.bn == 256) return run<256, false, 2, false, true>(a, pl, stream, why);
+    if (pl.bn == 128) return run<128, false, 2, false, true>(a, pl, stream, why);
+    return run<64, false, 2, false, true>(a, pl, stream, why);
   }
   if (pl.swap) return run<64, false, 2, true>(a, pl, stream, why);
   if (pl.bn == 256) return run<256, false, 2, false>(a, pl, stream, why);

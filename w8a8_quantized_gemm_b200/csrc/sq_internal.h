@@ -84,23 +84,51 @@ struct OutlierView {
 // Per-row smooth + quantize: q[r,k] = clamp(rne(src[r,k]*vec[k] * 127/a_r)), scale[r] = a_r/127.
 cudaError_t launch_quant_rows(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, const float* vec,
                               const OutlierView& ov, int8_t* q, float* scale, cudaStream_t stream);
-// Per-tensor: global absmax of src*vec into *gmax_bits (reset first), then quantize with it.
+// Per-tensor: global absmax of src*vec into *gmax_bits (reset first), then quantize with it;
+// with `clip` (device fp32 [1]) no maximum is taken and *clip is used instead.
 cudaError_t launch_quant_tensor(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, const float* vec,
-                                unsigned int* gmax_bits, int8_t* q, float* scale1, cudaStream_t stream);
+                                unsigned int* gmax_bits, int8_t* q, float* scale1, cudaStream_t stream,
+                                const float* clip = nullptr);
+// Asymmetric per-row: scale[r] = range/255, zero[r] = -128 - rne(lo * 255/range).
+cudaError_t launch_quant_rows_asym(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, const float* vec,
+                                   int8_t* q, float* scale, int32_t* zero, cudaStream_t stream);
 
 // ---- LLM.int8 outlier bookkeeping (sq_outlier.cu)
-cudaError_t launch_outlier_mask(const float* amax, int64_t K, float threshold, uint32_t* mask, int32_t* prefix,
-                                int32_t* idx, int32_t* count, uint32_t* mask_out, int32_t* count_out,
-                                cudaStream_t stream);
+// Outlier columns amax_j > threshold (threshold_dev, device fp32 [1], replaces the value when
+// given).
+cudaError_t launch_outlier_mask(const float* amax, int64_t K, float threshold, const float* threshold_dev,
+                                uint32_t* mask, int32_t* prefix, int32_t* idx, int32_t* count, uint32_t* mask_out,
+                                int32_t* count_out, cudaStream_t stream);
 // dst[r, c] = c < count ? src[r, idx[c]] : 0 for c < roundup(count, 64).
 cudaError_t launch_gather_columns(const uint16_t* src, int64_t rows, int64_t ld, const int32_t* idx,
                                   const int32_t* count, uint16_t* dst, int64_t ld_dst, cudaStream_t stream);
+
+// ---- variants (sq_variants.cu)
+// s <- max(s / max(s) * 127, 1e-5), inv_s = 1/s (one CTA).
+cudaError_t launch_normalize_scale(float* s, float* inv_s, int64_t K, cudaStream_t stream);
+// rowsum[n] = sum_k Wq[n,k].
+cudaError_t launch_row_sums(const int8_t* Wq, int64_t N, int64_t K, int32_t* rowsum, cudaStream_t stream);
+// LayerNorm (norm 0) / RMSNorm (norm 1) + smoothing + per-row quantization; K <= 16384.
+cudaError_t launch_norm_quant(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, int norm,
+                              const uint16_t* gamma, const uint16_t* beta, float eps, const float* vec, int8_t* q,
+                              float* scale, float* mean_rstd, cudaStream_t stream);
+// threshold = fp32(mean + k * std) over all elements; ws of mean_std_workspace_bytes(rows).
+size_t mean_std_workspace_bytes(int64_t rows);
+cudaError_t launch_mean_std_threshold(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, double k,
+                                      float* threshold, double* mean_std, void* ws, cudaStream_t stream);
+// *out = the element of 1-based rank `rank` of the ascending |src|; ws of abs_percentile_workspace_bytes().
+size_t abs_percentile_workspace_bytes();
+cudaError_t launch_abs_percentile(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, uint64_t rank,
+                                  float* out, void* ws, cudaStream_t stream);
 
 // ---- tensor-core GEMM (sq_gemm.cu)
 struct GemmArgs {
   const int8_t* Xq = nullptr;       // [M, K]
   const int8_t* Wq = nullptr;       // [N, K]
-  const float* x_scale = nullptr;   // [M]
+  const float* x_scale = nullptr;   // [M] (x_per_token) or [1]
+  bool x_per_token = true;
+  const int32_t* x_zero = nullptr;  // [M] asymmetric-activation zero points, or nullptr
+  const int32_t* w_rowsum = nullptr;// [N] sum_k Wq[n,k] (with x_zero)
   const float* w_scale = nullptr;   // [N] or [1]
   bool w_per_channel = true;
   const uint16_t* bias = nullptr;   // [N] bf16 or nullptr

@@ -20,7 +20,8 @@ constexpr int kMaskThreads = 1024;
 constexpr int kPrefetch = 8;
 
 __global__ void __launch_bounds__(kMaskThreads)
-outlier_mask_kernel(const float* __restrict__ amax, int64_t K, float threshold, uint32_t* __restrict__ mask,
+outlier_mask_kernel(const float* __restrict__ amax, int64_t K, float threshold_value,
+                    const float* __restrict__ threshold_dev, uint32_t* __restrict__ mask,
                     int32_t* __restrict__ prefix, int32_t* __restrict__ idx, int32_t* __restrict__ count,
                     uint32_t* __restrict__ mask_out, int32_t* __restrict__ count_out) {
   __shared__ int32_t warp_cnt[kMaskThreads / 32];
@@ -28,6 +29,7 @@ outlier_mask_kernel(const float* __restrict__ amax, int64_t K, float threshold, 
   __shared__ int32_t running;
   griddep_wait();
   griddep_launch_dependents();
+  const float threshold = threshold_dev != nullptr ? __ldg(threshold_dev) : threshold_value;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int64_t words = (K + 31) / 32;
@@ -107,11 +109,11 @@ __global__ void gather_columns_kernel(const uint16_t* __restrict__ src, int64_t 
 
 }  // namespace
 
-cudaError_t launch_outlier_mask(const float* amax, int64_t K, float threshold, uint32_t* mask, int32_t* prefix,
-                                int32_t* idx, int32_t* count, uint32_t* mask_out, int32_t* count_out,
-                                cudaStream_t stream) {
+cudaError_t launch_outlier_mask(const float* amax, int64_t K, float threshold, const float* threshold_dev,
+                                uint32_t* mask, int32_t* prefix, int32_t* idx, int32_t* count, uint32_t* mask_out,
+                                int32_t* count_out, cudaStream_t stream) {
   return launch_kernel(outlier_mask_kernel, dim3(1), dim3(kMaskThreads), 0, stream, false, amax, K, threshold,
-                       mask, prefix, idx, count, mask_out, count_out);
+                       threshold_dev, mask, prefix, idx, count, mask_out, count_out);
 }
 
 cudaError_t launch_gather_columns(const uint16_t* src, int64_t rows, int64_t ld, const int32_t* idx,

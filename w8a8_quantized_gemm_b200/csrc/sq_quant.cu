@@ -15,75 +15,25 @@
 // Arithmetic, all IEEE fp32 with no contraction: x' = x * vec[k] (__fmul_rn),
 // a = max|x'|, r = 127/a (__fdiv_rn), d = a/127 (__fdiv_rn),
 // q = clamp(__float2int_rn(x' * r), -128, 127) (round half to even).
+// Asymmetric rows ("量化基础与INT8" 非对称量化, over the range extended to contain 0):
+// lo = min(0, min x'), hi = max(0, max x'), range = hi - lo, r = 255/range, d = range/255,
+// z = -128 - rne(lo * r), q = clamp(rne(x' * r) + z, -128, 127).
 #include "sq_internal.h"
+#include "sq_rows.cuh"
 
 #include <algorithm>
 
 namespace sq {
 namespace {
 
-constexpr int kCta = 256;
+using namespace rows;
 
 // 16 skip bits for columns k..k+15 (k % 16 == 0).
 __device__ __forceinline__ uint32_t skip_bits16(const uint32_t* __restrict__ mask, int64_t k) {
   return (__ldg(mask + (k >> 5)) >> (k & 31)) & 0xFFFFu;
 }
 
-__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
-  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
-         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
-}
-
-__device__ __forceinline__ int q8(float x, float r) {
-  int q = __float2int_rn(__fmul_rn(x, r));
-  return min(127, max(-128, q));
-}
-
-__device__ __forceinline__ void store_q16(int8_t* dst, const float (&v)[16], float r) {
-  uint4 o;
-  o.x = pack4(q8(v[0], r), q8(v[1], r), q8(v[2], r), q8(v[3], r));
-  o.y = pack4(q8(v[4], r), q8(v[5], r), q8(v[6], r), q8(v[7], r));
-  o.z = pack4(q8(v[8], r), q8(v[9], r), q8(v[10], r), q8(v[11], r));
-  o.w = pack4(q8(v[12], r), q8(v[13], r), q8(v[14], r), q8(v[15], r));
-  *reinterpret_cast<uint4*>(dst) = o;
-}
-
-// Max over the TPR threads of one row group; every thread of the group gets the result.
-template <int TPR>
-__device__ __forceinline__ float group_max(float a, float* red /* [kCta/32] */) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-  if constexpr (TPR > 32) {
-    constexpr int kWarpsPerGroup = TPR / 32;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int g0 = (warp / kWarpsPerGroup) * kWarpsPerGroup;
-    if (lane == 0) red[warp] = a;
-    __syncthreads();
-    float t = red[g0];
-#pragma unroll
-    for (int w = 1; w < kWarpsPerGroup; ++w) t = fmaxf(t, red[g0 + w]);
-    __syncthreads();
-    a = t;
-  }
-  return a;
-}
-
-enum Mode { kPerRow = 0, kTensorMax = 1, kTensorQuant = 2 };
-
-__device__ __forceinline__ void raw16(const uint16_t* p, uint4 (&r)[2]) {
-  r[0] = __ldg(reinterpret_cast<const uint4*>(p));
-  r[1] = __ldg(reinterpret_cast<const uint4*>(p + 8));
-}
-
-__device__ __forceinline__ void widen16(const uint4 (&r)[2], float (&v)[16]) {
-  const uint32_t w[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    v[2 * i] = __uint_as_float(w[i] << 16);
-    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
+enum Mode { kPerRow = 0, kTensorMax = 1, kTensorQuant = 2, kAsym = 3 };
 
 // Zero the LLM.int8 outlier columns among k..k+15 (copying their bf16 values to the gathered
 // matrix when `gather`), then smooth with the thread's slice of the vector (if any).
@@ -121,7 +71,7 @@ template <int TPR, int CHUNKS, bool TWO_PASS, bool OUTLIERS, bool HAS_VEC, int M
 __global__ void __launch_bounds__(TPR > kCta ? TPR : kCta)
 quant_rows_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
                   const float* __restrict__ vec, OutlierView ov, int8_t* __restrict__ q,
-                  float* __restrict__ scale, unsigned int* __restrict__ gmax_bits) {
+                  float* __restrict__ scale, unsigned int* __restrict__ gmax_bits, int32_t* __restrict__ zero) {
   constexpr int kThreads = TPR > kCta ? TPR : kCta;
   griddep_wait();
   griddep_launch_dependents();
@@ -169,6 +119,7 @@ quant_rows_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
     const bool row_ok = row < rows;
     const uint16_t* srow = src + (row_ok ? row : 0) * ld;
     float a = 0.0f;
+    float lo = 0.0f;  // kAsym: a holds max(0, max x'), lo holds min(0, min x')
     float v[TWO_PASS ? 1 : CHUNKS][16];
     if constexpr (!TWO_PASS) {
 #pragma unroll
@@ -176,8 +127,16 @@ quant_rows_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
         const int64_t k = c * step + t * 16;
         if (row_ok && k < K) {
           finish_chunk<OUTLIERS, HAS_VEC>(raw[c], row, k, vs[HAS_VEC ? c : 0], ov, MODE != kTensorMax, v[c]);
+          if constexpr (MODE == kAsym) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[c][i]));
+            for (int i = 0; i < 16; ++i) {
+              a = fmaxf(a, v[c][i]);
+              lo = fminf(lo, v[c][i]);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[c][i]));
+          }
         }
       }
       // prefetch this thread's next row while the current one is reduced
@@ -203,18 +162,63 @@ quant_rows_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
           }
         }
         finish_chunk<OUTLIERS, HAS_VEC>(r, row, k, vv, ov, false, w);
+        if constexpr (MODE == kAsym) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(w[i]));
+          for (int i = 0; i < 16; ++i) {
+            a = fmaxf(a, w[i]);
+            lo = fminf(lo, w[i]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(w[i]));
+        }
       }
     }
 
     if constexpr (MODE == kTensorQuant) {
       a = __uint_as_float(*reinterpret_cast<volatile unsigned int*>(gmax_bits));
+    } else if constexpr (MODE == kAsym) {
+      a = group_max<TPR>(a, red);
+      lo = -group_max<TPR>(-lo, red);
     } else {
       a = group_max<TPR>(a, red);
     }
 
-    if constexpr (MODE == kTensorMax) {
+    if constexpr (MODE == kAsym) {
+      const float range = __fsub_rn(a, lo);
+      const float r = range > 0.0f ? __fdiv_rn(255.0f, range) : 0.0f;
+      const int z = -128 - __float2int_rn(__fmul_rn(lo, r));
+      if (row_ok) {
+        if (t == 0) {
+          scale[row] = __fdiv_rn(range, 255.0f);
+          zero[row] = z;
+        }
+        int8_t* qrow = q + row * K;
+        if constexpr (!TWO_PASS) {
+#pragma unroll
+          for (int c = 0; c < CHUNKS; ++c) {
+            const int64_t k = c * step + t * 16;
+            if (k < K) store_q16z(qrow + k, v[c], r, z);
+          }
+        } else {
+          for (int64_t k = t * 16; k < K; k += step) {
+            uint4 rr[2];
+            float w[16], vv[16];
+            raw16(srow + k, rr);
+            if constexpr (HAS_VEC) {
+              const float4* p4 = reinterpret_cast<const float4*>(vec + k);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float4 f = __ldg(p4 + i);
+                vv[4 * i] = f.x; vv[4 * i + 1] = f.y; vv[4 * i + 2] = f.z; vv[4 * i + 3] = f.w;
+              }
+            }
+            finish_chunk<false, HAS_VEC>(rr, row, k, vv, ov, false, w);
+            store_q16z(qrow + k, w, r, z);
+          }
+        }
+      }
+    } else if constexpr (MODE == kTensorMax) {
       if (t == 0 && row_ok) atomicMax(gmax_bits, __float_as_uint(a));
     } else {
       const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
@@ -284,7 +288,8 @@ int64_t resident_grid(Kernel kernel, int threads, int64_t groups, int& per_sm_ca
 
 template <int TPR, int CHUNKS, bool TWO_PASS, bool OUTLIERS, int MODE>
 cudaError_t launch_t(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, const float* vec,
-                     const OutlierView& ov, int8_t* q, float* scale, unsigned int* gmax, cudaStream_t stream) {
+                     const OutlierView& ov, int8_t* q, float* scale, unsigned int* gmax, int32_t* zero,
+                     cudaStream_t stream) {
   constexpr int kThreads = TPR > kCta ? TPR : kCta;
   constexpr int kGroups = kThreads / TPR;
   const int64_t groups = (rows + kGroups - 1) / kGroups;
@@ -293,13 +298,13 @@ cudaError_t launch_t(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, c
     auto kernel = quant_rows_kernel<TPR, CHUNKS, TWO_PASS, OUTLIERS, true, MODE>;
     const int64_t blocks = resident_grid(kernel, kThreads, groups, per_sm);
     return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, stream, false, src, rows,
-                         K, ld, vec, ov, q, scale, gmax);
+                         K, ld, vec, ov, q, scale, gmax, zero);
   }
   static int per_sm = 0;
   auto kernel = quant_rows_kernel<TPR, CHUNKS, TWO_PASS, OUTLIERS, false, MODE>;
   const int64_t blocks = resident_grid(kernel, kThreads, groups, per_sm);
   return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, stream, false, src, rows, K,
-                       ld, vec, ov, q, scale, gmax);
+                       ld, vec, ov, q, scale, gmax, zero);
 }
 
 // Shape dispatch: one 16-element chunk per thread up to K = 4096 (a row over up to 256
@@ -308,14 +313,22 @@ cudaError_t launch_t(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, c
 // K = 4096, two chunks at K = 8192.)
 template <bool OUTLIERS, int MODE>
 cudaError_t dispatch(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, const float* vec,
-                     const OutlierView& ov, int8_t* q, float* scale, unsigned int* gmax, cudaStream_t stream) {
-  if (K <= 512) return launch_t<32, 1, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
-  if (K <= 1024) return launch_t<64, 1, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
-  if (K <= 2048) return launch_t<128, 1, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
-  if (K <= 4096) return launch_t<256, 1, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
-  if (K <= 8192) return launch_t<256, 2, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
-  if (K <= 16384) return launch_t<512, 2, false, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
-  return launch_t<512, 1, true, OUTLIERS, MODE>(src, rows, K, ld, vec, ov, q, scale, gmax, stream);
+                     const OutlierView& ov, int8_t* q, float* scale, unsigned int* gmax, cudaStream_t stream,
+                     int32_t* zero = nullptr) {
+  if (K <= 512) return launch_t<32, 1, false, OUTLIERS, MODE>(
+      src, rows, K, ld, vec, ov, q, scale, gmax, zero, stream);
+  if (K <= 1024) return launch_t<64, 1, false, OUTLIERS, MODE>(
+      src, rows, K, ld, vec, ov, q, scale, gmax, zero, stream);
+  if (K <= 2048) return launch_t<128, 1, false, OUTLIERS, MODE>(
+      src, rows, K, ld, vec, ov, q, scale, gmax, zero, stream);
+  if (K <= 4096) return launch_t<256, 1, false, OUTLIERS, MODE>(
+      src, rows, K, ld, vec, ov, q, scale, gmax, zero, stream);
+  if (K <= 8192) return launch_t<256, 2, false, OUTLIERS, MODE>(
+      src, rows, K, ld, vec, ov, q, scale, gmax, zero, stream);
+  if (K <= 16384) return launch_t<512, 2, false, OUTLIERS, MODE>(
+      src, rows, K, ld, vec, ov, q, scale, gmax, zero, stream);
+  return launch_t<512, 1, true, OUTLIERS, MODE>(
+      src, rows, K, ld, vec, ov, q, scale, gmax, zero, stream);
 }
 
 }  // namespace
@@ -327,13 +340,24 @@ cudaError_t launch_quant_rows(const uint16_t* src, int64_t rows, int64_t K, int6
 }
 
 cudaError_t launch_quant_tensor(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, const float* vec,
-                                unsigned int* gmax_bits, int8_t* q, float* scale1, cudaStream_t stream) {
+                                unsigned int* gmax_bits, int8_t* q, float* scale1, cudaStream_t stream,
+                                const float* clip) {
+  OutlierView none;
+  if (clip != nullptr) {
+    // a calibrated value: one pass, the kernel reads the maximum from `clip`
+    unsigned int* c = reinterpret_cast<unsigned int*>(const_cast<float*>(clip));
+    return dispatch<false, kTensorQuant>(src, rows, K, ld, vec, none, q, scale1, c, stream);
+  }
   cudaError_t e = launch_zero_words(gmax_bits, 1, stream);
   if (e != cudaSuccess) return e;
-  OutlierView none;
   e = dispatch<false, kTensorMax>(src, rows, K, ld, vec, none, nullptr, nullptr, gmax_bits, stream);
   if (e != cudaSuccess) return e;
   return dispatch<false, kTensorQuant>(src, rows, K, ld, vec, none, q, scale1, gmax_bits, stream);
+}
+
+cudaError_t launch_quant_rows_asym(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, const float* vec,
+                                   int8_t* q, float* scale, int32_t* zero, cudaStream_t stream) {
+  return dispatch<false, kAsym>(src, rows, K, ld, vec, OutlierView{}, q, scale, nullptr, stream, zero);
 }
 
 }  // namespace sq

@@ -1,0 +1,104 @@
+// Device helpers shared by the row kernels (quantization of rows, fused normalisation):
+// 16-element bf16 loads, int8 packing with round-half-to-even, and reductions over the
+// TPR threads that own one row.
+#pragma once
+#include <cstdint>
+
+namespace sq {
+namespace rows {
+
+constexpr int kCta = 256;  // minimum CTA size of the row kernels
+
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
+         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
+}
+
+__device__ __forceinline__ int q8(float x, float r) {
+  int q = __float2int_rn(__fmul_rn(x, r));
+  return min(127, max(-128, q));
+}
+
+__device__ __forceinline__ void store_q16(int8_t* dst, const float (&v)[16], float r) {
+  uint4 o;
+  o.x = pack4(q8(v[0], r), q8(v[1], r), q8(v[2], r), q8(v[3], r));
+  o.y = pack4(q8(v[4], r), q8(v[5], r), q8(v[6], r), q8(v[7], r));
+  o.z = pack4(q8(v[8], r), q8(v[9], r), q8(v[10], r), q8(v[11], r));
+  o.w = pack4(q8(v[12], r), q8(v[13], r), q8(v[14], r), q8(v[15], r));
+  *reinterpret_cast<uint4*>(dst) = o;
+}
+
+// Codes of 16 values with a zero point: clamp(rne(v * r) + z, -128, 127).
+__device__ __forceinline__ int q8z(float x, float r, int z) {
+  const int q = __float2int_rn(__fmul_rn(x, r)) + z;
+  return min(127, max(-128, q));
+}
+
+__device__ __forceinline__ void store_q16z(int8_t* dst, const float (&v)[16], float r, int z) {
+  uint4 o;
+  o.x = pack4(q8z(v[0], r, z), q8z(v[1], r, z), q8z(v[2], r, z), q8z(v[3], r, z));
+  o.y = pack4(q8z(v[4], r, z), q8z(v[5], r, z), q8z(v[6], r, z), q8z(v[7], r, z));
+  o.z = pack4(q8z(v[8], r, z), q8z(v[9], r, z), q8z(v[10], r, z), q8z(v[11], r, z));
+  o.w = pack4(q8z(v[12], r, z), q8z(v[13], r, z), q8z(v[14], r, z), q8z(v[15], r, z));
+  *reinterpret_cast<uint4*>(dst) = o;
+}
+
+// Max over the TPR threads of one row group; every thread of the group gets the result.
+template <int TPR>
+__device__ __forceinline__ float group_max(float a, float* red /* [kCta/32] */) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if constexpr (TPR > 32) {
+    constexpr int kWarpsPerGroup = TPR / 32;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g0 = (warp / kWarpsPerGroup) * kWarpsPerGroup;
+    if (lane == 0) red[warp] = a;
+    __syncthreads();
+    float t = red[g0];
+#pragma unroll
+    for (int w = 1; w < kWarpsPerGroup; ++w) t = fmaxf(t, red[g0 + w]);
+    __syncthreads();
+    a = t;
+  }
+  return a;
+}
+
+__device__ __forceinline__ void raw16(const uint16_t* p, uint4 (&r)[2]) {
+  r[0] = __ldg(reinterpret_cast<const uint4*>(p));
+  r[1] = __ldg(reinterpret_cast<const uint4*>(p + 8));
+}
+
+__device__ __forceinline__ void widen16(const uint4 (&r)[2], float (&v)[16]) {
+  const uint32_t w[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// Sum over the TPR threads of one row group in fp64 (fixed order: butterfly within the warp,
+// then the warps of the group in index order); every thread of the group gets the result.
+template <int TPR>
+__device__ __forceinline__ double group_sum(double a, double* red /* [CTA threads / 32] */) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = __dadd_rn(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if constexpr (TPR > 32) {
+    constexpr int kWarpsPerGroup = TPR / 32;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g0 = (warp / kWarpsPerGroup) * kWarpsPerGroup;
+    if (lane == 0) red[warp] = a;
+    __syncthreads();
+    double t = red[g0];
+#pragma unroll
+    for (int w = 1; w < kWarpsPerGroup; ++w) t = __dadd_rn(t, red[g0 + w]);
+    __syncthreads();
+    a = t;
+  }
+  return a;
+}
+
+}  // namespace rows
+}  // namespace sq

@@ -1,0 +1,479 @@
+// Kernels of the variants around the W8A8 layer:
+//   - normalisation of the smoothing factors,
+//     "SmoothQuant量化实战：W8A8推理部署与单节点530B模型落地" §3.3 (s / s.max() * 127, clamp 1e-5);
+//   - LayerNorm / RMSNorm fused with smoothing and per-token quantization, the same page
+//     §4.2 and §4.5 second detail (the smoothing folds into the LayerNorm output);
+//   - mean + k*std outlier threshold over the activations, "LLM.int8()技术解析" §3.1
+//     (threshold = mu + 6 sigma) and "从自动驾驶芯片到大语言模型INT8量化训练实战解析" §2.1;
+//   - nearest-rank percentile of |X| for static calibration, the page on choosing
+//     quantization precision ("大语言模型轻量化与量化精度") §3.2 (percentile 99.99);
+//   - row sums of the int8 weight (zero-point correction of asymmetric activations,
+//     "量化基础与INT8" 非对称量化).
+// All of them are HBM-bound passes over bf16 / int8 matrices with 16-byte loads; the
+// reductions that feed a floating-point decision are summed in fp64 in a fixed order, so
+// every result is deterministic run to run.
+#include "sq_internal.h"
+#include "sq_rows.cuh"
+
+#include <algorithm>
+#include <atomic>
+
+namespace sq {
+namespace {
+
+using namespace rows;
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+// ------------------------------------------------------------------ smoothing factors
+// One CTA: smax = max_j s_j, then s_j <- max((s_j / smax) * 127, 1e-5), inv_s_j = 1/s_j.
+__global__ void __launch_bounds__(1024) normalize_scale_kernel(float* __restrict__ s, float* __restrict__ inv_s,
+                                                               int64_t K) {
+  griddep_wait();
+  griddep_launch_dependents();
+  __shared__ float red[32];
+  float m = 0.0f;
+  for (int64_t j = threadIdx.x; j < K; j += blockDim.x) m = fmaxf(m, s[j]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float smax = red[0];
+  for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) smax = fmaxf(smax, red[w]);
+  for (int64_t j = threadIdx.x; j < K; j += blockDim.x) {
+    const float t = fmaxf(__fmul_rn(__fdiv_rn(s[j], smax), 127.0f), 1e-5f);
+    s[j] = t;
+    inv_s[j] = __fdiv_rn(1.0f, t);
+  }
+}
+
+// ------------------------------------------------------------------ weight row sums
+// One warp per row: rowsum[n] = sum_k Wq[n,k] (16-byte loads, dp4a against ones).
+__global__ void __launch_bounds__(256) row_sums_kernel(const int8_t* __restrict__ Wq, int64_t N, int64_t K,
+                                                       int32_t* __restrict__ rowsum) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); n < N; n += warps) {
+    const int4* row = reinterpret_cast<const int4*>(Wq + n * K);
+    int acc = 0;
+    for (int64_t v = lane; v < K / 16; v += 32) {
+      const int4 w = __ldg(row + v);
+      acc = __dp4a(w.x, 0x01010101, acc);
+      acc = __dp4a(w.y, 0x01010101, acc);
+      acc = __dp4a(w.z, 0x01010101, acc);
+      acc = __dp4a(w.w, 0x01010101, acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) rowsum[n] = acc;
+  }
+}
+
+// ------------------------------------------------------------------ fused normalisation
+// Row groups of TPR threads walk the rows with a grid stride (as the row quantization
+// kernel does); a thread owns 16 consecutive columns per chunk and keeps its row values in
+// registers between the statistics, the absmax and the quantization, and prefetches its
+// next row. With one chunk per thread its slices of gamma, beta and inv_s stay in
+// registers for all its rows; with two they are re-read per row (L1 hits) to keep the
+// register count within the launch bound.
+template <int TPR, int CHUNKS>
+__global__ void __launch_bounds__(TPR > kCta ? TPR : kCta)
+norm_quant_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int norm,
+                  const uint16_t* __restrict__ gamma, const uint16_t* __restrict__ beta, float eps,
+                  const float* __restrict__ vec, int8_t* __restrict__ q, float* __restrict__ scale,
+                  float* __restrict__ mean_rstd) {
+  constexpr int kThreads = TPR > kCta ? TPR : kCta;
+  constexpr int kGroups = kThreads / TPR;
+  griddep_wait();
+  griddep_launch_dependents();
+  __shared__ float redf[kThreads / 32];
+  __shared__ double redd[kThreads / 32];
+  const int g = threadIdx.x / TPR;
+  const int t = threadIdx.x % TPR;
+  const int64_t step = static_cast<int64_t>(TPR) * 16;
+  const int64_t row_stride = static_cast<int64_t>(gridDim.x) * kGroups;
+  const bool layer = (norm == 0);
+  const bool has_beta = beta != nullptr;
+  const bool has_vec = vec != nullptr;
+
+  constexpr bool kResident = CHUNKS == 1;
+  // gamma, beta (0 when absent) and inv_s (1 when absent) of columns k..k+15; columns past
+  // K get gamma = 0, so their y is 0 and they do not enter the absmax
+  auto load_vectors = [&](int64_t k, float (&g16)[16], float (&b16)[16], float (&v16)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      g16[i] = 0.0f;
+      b16[i] = 0.0f;
+      v16[i] = 1.0f;
+    }
+    if (k < K) {
+      uint4 r[2];
+      raw16(gamma + k, r);
+      widen16(r, g16);
+      if (has_beta) {
+        raw16(beta + k, r);
+        widen16(r, b16);
+      }
+      if (has_vec) {
+        const float4* p4 = reinterpret_cast<const float4*>(vec + k);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 f = __ldg(p4 + i);
+          v16[4 * i] = f.x;
+          v16[4 * i + 1] = f.y;
+          v16[4 * i + 2] = f.z;
+          v16[4 * i + 3] = f.w;
+        }
+      }
+    }
+  };
+  float gs[1][16], bs[1][16], vs[1][16];  // this thread's chunk (the only one when resident)
+  if constexpr (kResident) load_vectors(t * 16, gs[0], bs[0], vs[0]);
+
+  uint4 raw[CHUNKS][2];
+  int64_t row = static_cast<int64_t>(blockIdx.x) * kGroups + g;
+  if (row < rows) {
+#pragma unroll
+    for (int c = 0; c < CHUNKS; ++c) {
+      const int64_t k = c * step + t * 16;
+      if (k < K) raw16(src + row * ld + k, raw[c]);
+    }
+  }
+
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kGroups; base < rows; base += row_stride, row += row_stride) {
+    const bool row_ok = row < rows;
+    float x[CHUNKS][16];
+#pragma unroll
+    for (int c = 0; c < CHUNKS; ++c) {
+      const int64_t k = c * step + t * 16;
+      if (row_ok && k < K) {
+        widen16(raw[c], x[c]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[c][i] = 0.0f;
+      }
+    }
+    // prefetch this thread's next row while the current one is reduced
+    const int64_t nrow = row + row_stride;
+    if (nrow < rows) {
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) {
+        const int64_t k = c * step + t * 16;
+        if (k < K) raw16(src + nrow * ld + k, raw[c]);
+      }
+    }
+    // row statistics in fp64 (absent columns hold 0 and are skipped in the deviations)
+    float mean_f = 0.0f;
+    double ss = 0.0;
+    if (layer) {
+      double s1 = 0.0;
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) s1 = __dadd_rn(s1, static_cast<double>(x[c][i]));
+      const double mean = __ddiv_rn(group_sum<TPR>(s1, redd), static_cast<double>(K));
+      mean_f = __double2float_rn(mean);
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) {
+        if (c * step + t * 16 < K) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const double dv = __dsub_rn(static_cast<double>(x[c][i]), mean);
+            ss = __dadd_rn(ss, __dmul_rn(dv, dv));
+          }
+        }
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const double dv = static_cast<double>(x[c][i]);
+          ss = __dadd_rn(ss, __dmul_rn(dv, dv));
+        }
+    }
+    const double m2 = __ddiv_rn(group_sum<TPR>(ss, redd), static_cast<double>(K));
+    const float rstd_f = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(m2, static_cast<double>(eps)))));
+    // y = ((x - mean) * rstd) * gamma + beta, x' = y * inv_s, absmax
+    float a = 0.0f;
+#pragma unroll
+    for (int c = 0; c < CHUNKS; ++c) {
+      if constexpr (!kResident) load_vectors(c * step + t * 16, gs[0], bs[0], vs[0]);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float y = layer ? __fmul_rn(__fsub_rn(x[c][i], mean_f), rstd_f) : __fmul_rn(x[c][i], rstd_f);
+        y = __fmul_rn(y, gs[0][i]);
+        if (has_beta) y = __fadd_rn(y, bs[0][i]);
+        if (has_vec) y = __fmul_rn(y, vs[0][i]);
+        x[c][i] = y;
+        a = fmaxf(a, fabsf(y));
+      }
+    }
+    a = group_max<TPR>(a, redf);
+    const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+    if (row_ok) {
+      if (t == 0) {
+        scale[row] = __fdiv_rn(a, 127.0f);
+        if (mean_rstd != nullptr) {
+          mean_rstd[2 * row] = mean_f;
+          mean_rstd[2 * row + 1] = rstd_f;
+        }
+      }
+      int8_t* qrow = q + row * K;
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) {
+        const int64_t k = c * step + t * 16;
+        if (k < K) store_q16(qrow + k, x[c], r);
+      }
+    }
+  }
+}
+
+template <int TPR, int CHUNKS>
+cudaError_t launch_norm_t(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, int norm, const uint16_t* gamma,
+                          const uint16_t* beta, float eps, const float* vec, int8_t* q, float* scale,
+                          float* mean_rstd, cudaStream_t stream) {
+  constexpr int kThreads = TPR > kCta ? TPR : kCta;
+  constexpr int kGroups = kThreads / TPR;
+  auto kernel = norm_quant_kernel<TPR, CHUNKS>;
+  static int per_sm = 0;
+  if (per_sm <= 0) {
+    int v = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, kThreads, 0) != cudaSuccess || v < 1) v = 1;
+    per_sm = v;
+  }
+  const int64_t groups = (rows + kGroups - 1) / kGroups;
+  const int64_t blocks = std::min<int64_t>(groups, static_cast<int64_t>(sm_count()) * per_sm);
+  return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, stream, false, src, rows, K,
+                       ld, norm, gamma, beta, eps, vec, q, scale, mean_rstd);
+}
+
+// ------------------------------------------------------------------ mean / std threshold
+constexpr int kStatThreads = 256;
+
+// partial[b] = sum of the elements of CTA b's rows (fp64, fixed order).
+__global__ void __launch_bounds__(kStatThreads)
+sum_partials_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int64_t rows_per_cta,
+                    const double* __restrict__ mean_in, double* __restrict__ partial) {
+  griddep_wait();
+  griddep_launch_dependents();
+  __shared__ double red[kStatThreads / 32];
+  // second pass: sum of squared deviations from the mean of the first
+  const bool dev = mean_in != nullptr;
+  const double mean = dev ? *mean_in : 0.0;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows_per_cta;
+  const int64_t r1 = min(rows, r0 + rows_per_cta);
+  const int64_t vecs = K / 8;
+  double acc = 0.0;
+  for (int64_t r = r0; r < r1; ++r) {
+    const uint4* p = reinterpret_cast<const uint4*>(src + r * ld);
+    for (int64_t v = threadIdx.x; v < vecs; v += kStatThreads) {
+      const uint4 w = __ldg(p + v);
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const double lo = static_cast<double>(__uint_as_float(u[i] << 16));
+        const double hi = static_cast<double>(__uint_as_float(u[i] & 0xFFFF0000u));
+        if (dev) {
+          const double a = __dsub_rn(lo, mean), b = __dsub_rn(hi, mean);
+          acc = __dadd_rn(acc, __dmul_rn(a, a));
+          acc = __dadd_rn(acc, __dmul_rn(b, b));
+        } else {
+          acc = __dadd_rn(acc, lo);
+          acc = __dadd_rn(acc, hi);
+        }
+      }
+    }
+  }
+  acc = group_sum<kStatThreads>(acc, red);
+  if (threadIdx.x == 0) partial[blockIdx.x] = acc;
+}
+
+// One CTA: total = sum of the G partials in a fixed order; writes total / divisor to *out.
+__global__ void __launch_bounds__(kStatThreads)
+reduce_partials_kernel(const double* __restrict__ partial, int G, double divisor, double* __restrict__ out) {
+  griddep_wait();
+  griddep_launch_dependents();
+  __shared__ double red[kStatThreads / 32];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < G; i += kStatThreads) acc = __dadd_rn(acc, partial[i]);
+  acc = group_sum<kStatThreads>(acc, red);
+  if (threadIdx.x == 0) *out = __ddiv_rn(acc, divisor);
+}
+
+// threshold = fp32(mean + k * sqrt(var)), var = ss / (n - 1) already in stats[1].
+__global__ void threshold_kernel(const double* __restrict__ stats, double k, float* __restrict__ threshold,
+                                 double* __restrict__ mean_std) {
+  griddep_wait();
+  griddep_launch_dependents();
+  if (threadIdx.x != 0) return;
+  const double mean = stats[0];
+  const double sd = __dsqrt_rn(stats[1]);
+  *threshold = __double2float_rn(__dadd_rn(mean, __dmul_rn(k, sd)));
+  if (mean_std != nullptr) {
+    mean_std[0] = mean;
+    mean_std[1] = sd;
+  }
+}
+
+// ------------------------------------------------------------------ percentile
+constexpr int kBins = 1 << 15;  // bf16 magnitudes (sign dropped)
+constexpr int kHistThreads = 1024;
+
+// Per-CTA histogram of |x| bit patterns in shared memory, added into the global one.
+__global__ void __launch_bounds__(kHistThreads)
+abs_hist_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
+                unsigned long long* __restrict__ hist) {
+  griddep_wait();
+  griddep_launch_dependents();
+  extern __shared__ uint32_t sh[];
+  for (int b = threadIdx.x; b < kBins; b += kHistThreads) sh[b] = 0u;
+  __syncthreads();
+  const int64_t vecs_per_row = K / 8;
+  const int64_t total = rows * vecs_per_row;
+  for (int64_t v = static_cast<int64_t>(blockIdx.x) * kHistThreads + threadIdx.x; v < total;
+       v += static_cast<int64_t>(gridDim.x) * kHistThreads) {
+    const int64_t r = v / vecs_per_row;
+    const int64_t c = v - r * vecs_per_row;
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + r * ld) + c);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      atomicAdd(&sh[u[i] & 0x7FFFu], 1u);
+      atomicAdd(&sh[(u[i] >> 16) & 0x7FFFu], 1u);
+    }
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < kBins; b += kHistThreads)
+    if (sh[b] != 0u) atomicAdd(hist + b, static_cast<unsigned long long>(sh[b]));
+}
+
+// One CTA of 1024 threads, 32 bins each: the bin holding the element of 1-based rank `rank`
+// (the first bin whose inclusive cumulative count reaches it) gives the value.
+__global__ void __launch_bounds__(kHistThreads)
+select_rank_kernel(const unsigned long long* __restrict__ hist, unsigned long long rank, float* __restrict__ out) {
+  griddep_wait();
+  griddep_launch_dependents();
+  constexpr int kPer = kBins / kHistThreads;
+  __shared__ unsigned long long part[kHistThreads];
+  const int t = threadIdx.x;
+  unsigned long long mine = 0;
+#pragma unroll 4
+  for (int i = 0; i < kPer; ++i) mine += hist[t * kPer + i];
+  part[t] = mine;
+  __syncthreads();
+  // inclusive scan over the 1024 partial counts (Hillis-Steele, exact integers)
+  for (int o = 1; o < kHistThreads; o <<= 1) {
+    const unsigned long long add = t >= o ? part[t - o] : 0ull;
+    __syncthreads();
+    part[t] += add;
+    __syncthreads();
+  }
+  const unsigned long long before = t > 0 ? part[t - 1] : 0ull;
+  if (before < rank && part[t] >= rank) {
+    unsigned long long run = before;
+    for (int i = 0; i < kPer; ++i) {
+      run += hist[t * kPer + i];
+      if (run >= rank) {
+        *out = __uint_as_float(static_cast<uint32_t>(t * kPer + i) << 16);
+        break;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_normalize_scale(float* s, float* inv_s, int64_t K, cudaStream_t stream) {
+  return launch_kernel(normalize_scale_kernel, dim3(1), dim3(1024), 0, stream, false, s, inv_s, K);
+}
+
+cudaError_t launch_row_sums(const int8_t* Wq, int64_t N, int64_t K, int32_t* rowsum, cudaStream_t stream) {
+  const int64_t blocks = std::min<int64_t>((N + 7) / 8, static_cast<int64_t>(sm_count()) * 8);
+  return launch_kernel(row_sums_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream, false, Wq, N, K,
+                       rowsum);
+}
+
+cudaError_t launch_norm_quant(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, int norm,
+                              const uint16_t* gamma, const uint16_t* beta, float eps, const float* vec, int8_t* q,
+                              float* scale, float* mean_rstd, cudaStream_t stream) {
+#define SQ_NORM_ARGS src, rows, K, ld, norm, gamma, beta, eps, vec, q, scale, mean_rstd, stream
+  if (K <= 512) return launch_norm_t<32, 1>(SQ_NORM_ARGS);
+  if (K <= 1024) return launch_norm_t<64, 1>(SQ_NORM_ARGS);
+  if (K <= 2048) return launch_norm_t<128, 1>(SQ_NORM_ARGS);
+  if (K <= 4096) return launch_norm_t<256, 1>(SQ_NORM_ARGS);
+  if (K <= 8192) return launch_norm_t<256, 2>(SQ_NORM_ARGS);
+  return launch_norm_t<512, 2>(SQ_NORM_ARGS);
+#undef SQ_NORM_ARGS
+}
+
+int64_t mean_std_ctas(int64_t rows) { return std::min<int64_t>(rows, 1024); }
+
+size_t mean_std_workspace_bytes(int64_t rows) {
+  // two partial arrays of G doubles and two statistics
+  return sizeof(double) * (2 * static_cast<size_t>(mean_std_ctas(rows)) + 2);
+}
+
+cudaError_t launch_mean_std_threshold(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, double k,
+                                      float* threshold, double* mean_std, void* ws, cudaStream_t stream) {
+  const int64_t G = mean_std_ctas(rows);
+  const int64_t rpc = (rows + G - 1) / G;
+  const int64_t ctas = (rows + rpc - 1) / rpc;
+  double* part1 = static_cast<double*>(ws);
+  double* part2 = part1 + G;
+  double* stats = part2 + G;  // [0] mean, [1] variance
+  const double n = static_cast<double>(rows) * static_cast<double>(K);
+  cudaError_t e = launch_kernel(sum_partials_kernel, dim3(static_cast<unsigned>(ctas)), dim3(kStatThreads), 0,
+                                stream, false, src, rows, K, ld, rpc, static_cast<const double*>(nullptr), part1);
+  if (e == cudaSuccess)
+    e = launch_kernel(reduce_partials_kernel, dim3(1), dim3(kStatThreads), 0, stream, false,
+                      static_cast<const double*>(part1), static_cast<int>(ctas), n, stats);
+  if (e == cudaSuccess)
+    e = launch_kernel(sum_partials_kernel, dim3(static_cast<unsigned>(ctas)), dim3(kStatThreads), 0, stream, false,
+                      src, rows, K, ld, rpc, static_cast<const double*>(stats), part2);
+  if (e == cudaSuccess)
+    e = launch_kernel(reduce_partials_kernel, dim3(1), dim3(kStatThreads), 0, stream, false,
+                      static_cast<const double*>(part2), static_cast<int>(ctas), n > 1.0 ? n - 1.0 : 1.0,
+                      stats + 1);
+  if (e == cudaSuccess)
+    e = launch_kernel(threshold_kernel, dim3(1), dim3(32), 0, stream, false, static_cast<const double*>(stats), k,
+                      threshold, mean_std);
+  return e;
+}
+
+size_t abs_percentile_workspace_bytes() { return sizeof(unsigned long long) * kBins; }
+
+cudaError_t launch_abs_percentile(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, uint64_t rank,
+                                  float* out, void* ws, cudaStream_t stream) {
+  unsigned long long* hist = static_cast<unsigned long long*>(ws);
+  cudaError_t e = launch_zero_words(reinterpret_cast<uint32_t*>(hist), 2 * static_cast<int64_t>(kBins), stream);
+  static std::atomic<uint64_t> attr_done{0};  // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t bit = 1ull << (dev & 63);
+  const size_t smem = sizeof(uint32_t) * kBins;
+  if (e == cudaSuccess && !(attr_done.load() & bit)) {
+    e = cudaFuncSetAttribute(abs_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e == cudaSuccess) attr_done.fetch_or(bit);
+  }
+  if (e == cudaSuccess) {
+    const int64_t vecs = rows * (K / 8);
+    const int64_t blocks =
+        std::max<int64_t>(1, std::min<int64_t>(sm_count(), (vecs + kHistThreads - 1) / kHistThreads));
+    e = launch_kernel(abs_hist_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kHistThreads), smem, stream, false,
+                      src, rows, K, ld, hist);
+  }
+  if (e == cudaSuccess)
+    e = launch_kernel(select_rank_kernel, dim3(1), dim3(kHistThreads), 0, stream, false,
+                      static_cast<const unsigned long long*>(hist), static_cast<unsigned long long>(rank), out);
+  return e;
+}
+
+}  // namespace sq

@@ -20,6 +20,8 @@ SQ_OK, SQ_ERR_INVALID, SQ_ERR_ALIGN, SQ_ERR_CUDA, SQ_ERR_TIMEOUT, SQ_ERR_WORKSPA
     0, -1, -2, -3, -4, -5, -6
 SQ_PER_TENSOR, SQ_PER_CHANNEL = 0, 1
 SQ_OP_SMOOTH_QUANT_WEIGHT, SQ_OP_INT8_GEMM_DEQUANT, SQ_OP_LLMINT8 = 1, 2, 3
+SQ_OP_QUANT_ACT_PER_TENSOR, SQ_OP_MEAN_STD_THRESHOLD, SQ_OP_ABS_PERCENTILE = 4, 5, 6
+SQ_NORM_LAYER, SQ_NORM_RMS = 0, 1
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python -m w8a8_quantized_gemm_b200.build`")
@@ -34,6 +36,16 @@ _SIGS = {
     "sq_int8_gemm_dequant": ([_p, _p, _p, _p, _i32, _p, _p, _i64, _i64, _i64, _p, _p, _sz, _p], _i32),
     "llmint8_decomposed_linear": ([_p, _p, _p, _p, _f32, _p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _sz, _p], _i32),
     "sq_smooth_quant_weight_noalloc": ([_p, _i64, _i64, _i64, _p, _i32, _p, _p, _p], _i32),
+    "sq_quant_act_per_tensor": ([_p, _i64, _i64, _i64, _p, _p, _p, _p, _p, _sz, _p], _i32),
+    "sq_smooth_scale_ex": ([_p, _p, _i64, _i64, _i64, _f32, _i32, _p, _p, _p], _i32),
+    "sq_int8_gemm_dequant_ex": ([_p, _p, _p, _i32, _p, _p, _i32, _p, _p, _p, _i64, _i64, _i64, _p, _p, _sz, _p],
+                                _i32),
+    "sq_norm_smooth_quant": ([_p, _i64, _i64, _i64, _i32, _p, _p, _f32, _p, _p, _p, _p, _p], _i32),
+    "sq_act_mean_std_threshold": ([_p, _i64, _i64, _i64, C.c_double, _p, _p, _p, _sz, _p], _i32),
+    "llmint8_decomposed_linear_ex": ([_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _sz, _p], _i32),
+    "sq_act_abs_percentile": ([_p, _i64, _i64, _i64, C.c_double, _p, _p, _sz, _p], _i32),
+    "sq_quant_act_per_token_asym": ([_p, _i64, _i64, _i64, _p, _p, _p, _p, _p], _i32),
+    "sq_weight_row_sums": ([_p, _i64, _i64, _p, _p], _i32),
     "sq_workspace_size": ([_i32, _i64, _i64, _i64], _sz),
     "sq_last_error": ([], C.c_char_p),
     "sq_sync_status": ([_p], _i32),
@@ -181,6 +193,106 @@ def llmint8_decomposed_linear(X, W, Wq, w_scale, threshold: float, bias, Y, mask
         _ptr(n_outliers_out, torch.int32, "n_outliers_out"), _ptr(acc_out, torch.int32, "acc_out"), wsp, wsb,
         _stream(stream)))
     return Y
+
+
+# ---------------------------------------------------------------- variants
+def sq_quant_act_per_tensor(X, inv_s, Xq, x_scale, clip=None, ws=None, stream=None):
+    """Per-tensor activation scale: dynamic (clip None, needs ws) or the calibrated *clip."""
+    torch = _torch()
+    M, K = X.shape
+    wsp, wsb = _ws(ws)
+    _check(_lib.sq_quant_act_per_tensor(_ptr(X, torch.bfloat16, "X", True), M, K, X.stride(0),
+                                        _ptr(inv_s, torch.float32, "inv_s"), _ptr(clip, torch.float32, "clip"),
+                                        _ptr(Xq, torch.int8, "Xq"), _ptr(x_scale, torch.float32, "x_scale"), wsp, wsb,
+                                        _stream(stream)))
+    return Xq, x_scale
+
+
+def sq_smooth_scale_ex(act_amax, W, alpha: float, normalize: bool, s, inv_s, stream=None):
+    torch = _torch()
+    N, K = W.shape
+    _check(_lib.sq_smooth_scale_ex(_ptr(act_amax, torch.float32, "act_amax"), _ptr(W, torch.bfloat16, "W", True), N,
+                                   K, W.stride(0), float(alpha), int(bool(normalize)), _ptr(s, torch.float32, "s"),
+                                   _ptr(inv_s, torch.float32, "inv_s"), _stream(stream)))
+    return s, inv_s
+
+
+def sq_int8_gemm_dequant_ex(Xq, Wq, x_scale, x_gran: int, x_zero, w_scale, w_gran: int, w_rowsum, bias, Y,
+                            acc_out=None, ws=None, stream=None):
+    torch = _torch()
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    wsp, wsb = _ws(ws)
+    _check(_lib.sq_int8_gemm_dequant_ex(
+        _ptr(Xq, torch.int8, "Xq"), _ptr(Wq, torch.int8, "Wq"), _ptr(x_scale, torch.float32, "x_scale"), int(x_gran),
+        _ptr(x_zero, torch.int32, "x_zero"), _ptr(w_scale, torch.float32, "w_scale"), int(w_gran),
+        _ptr(w_rowsum, torch.int32, "w_rowsum"), _ptr(bias, torch.bfloat16, "bias"), _ptr(Y, torch.bfloat16, "Y"),
+        M, N, K, _ptr(acc_out, torch.int32, "acc_out"), wsp, wsb, _stream(stream)))
+    return Y
+
+
+def sq_norm_smooth_quant(X, norm: int, gamma, beta, eps: float, inv_s, Xq, x_scale, mean_rstd=None, stream=None):
+    torch = _torch()
+    M, K = X.shape
+    _check(_lib.sq_norm_smooth_quant(_ptr(X, torch.bfloat16, "X", True), M, K, X.stride(0), int(norm),
+                                     _ptr(gamma, torch.bfloat16, "gamma"), _ptr(beta, torch.bfloat16, "beta"),
+                                     float(eps), _ptr(inv_s, torch.float32, "inv_s"), _ptr(Xq, torch.int8, "Xq"),
+                                     _ptr(x_scale, torch.float32, "x_scale"),
+                                     _ptr(mean_rstd, torch.float32, "mean_rstd"), _stream(stream)))
+    return Xq, x_scale
+
+
+def sq_act_mean_std_threshold(X, k: float, threshold, mean_std=None, ws=None, stream=None):
+    torch = _torch()
+    M, K = X.shape
+    wsp, wsb = _ws(ws)
+    _check(_lib.sq_act_mean_std_threshold(_ptr(X, torch.bfloat16, "X", True), M, K, X.stride(0), float(k),
+                                          _ptr(threshold, torch.float32, "threshold"),
+                                          _ptr(mean_std, torch.float64, "mean_std"), wsp, wsb, _stream(stream)))
+    return threshold
+
+
+def llmint8_decomposed_linear_ex(X, W, Wq, w_scale, threshold, bias, Y, mask_out=None, n_outliers_out=None,
+                                 acc_out=None, ws=None, stream=None):
+    """llmint8_decomposed_linear with the threshold in a device fp32 [1] tensor."""
+    torch = _torch()
+    M, K = X.shape
+    N = W.shape[0]
+    wsp, wsb = _ws(ws)
+    _check(_lib.llmint8_decomposed_linear_ex(
+        _ptr(X, torch.bfloat16, "X"), _ptr(W, torch.bfloat16, "W"), _ptr(Wq, torch.int8, "Wq"),
+        _ptr(w_scale, torch.float32, "w_scale"), _ptr(threshold, torch.float32, "threshold"),
+        _ptr(bias, torch.bfloat16, "bias"), _ptr(Y, torch.bfloat16, "Y"), M, N, K,
+        _ptr(mask_out, torch.int32, "mask_out"), _ptr(n_outliers_out, torch.int32, "n_outliers_out"),
+        _ptr(acc_out, torch.int32, "acc_out"), wsp, wsb, _stream(stream)))
+    return Y
+
+
+def sq_act_abs_percentile(X, p: float, out, ws=None, stream=None):
+    torch = _torch()
+    M, K = X.shape
+    wsp, wsb = _ws(ws)
+    _check(_lib.sq_act_abs_percentile(_ptr(X, torch.bfloat16, "X", True), M, K, X.stride(0), float(p),
+                                      _ptr(out, torch.float32, "out"), wsp, wsb, _stream(stream)))
+    return out
+
+
+def sq_quant_act_per_token_asym(X, inv_s, Xq, x_scale, x_zero, stream=None):
+    torch = _torch()
+    M, K = X.shape
+    _check(_lib.sq_quant_act_per_token_asym(_ptr(X, torch.bfloat16, "X", True), M, K, X.stride(0),
+                                            _ptr(inv_s, torch.float32, "inv_s"), _ptr(Xq, torch.int8, "Xq"),
+                                            _ptr(x_scale, torch.float32, "x_scale"),
+                                            _ptr(x_zero, torch.int32, "x_zero"), _stream(stream)))
+    return Xq, x_scale, x_zero
+
+
+def sq_weight_row_sums(Wq, rowsum, stream=None):
+    torch = _torch()
+    N, K = Wq.shape
+    _check(_lib.sq_weight_row_sums(_ptr(Wq, torch.int8, "Wq"), N, K, _ptr(rowsum, torch.int32, "rowsum"),
+                                   _stream(stream)))
+    return rowsum
 
 
 def sq_workspace_size(op: int, M: int, N: int, K: int) -> int:

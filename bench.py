@@ -364,6 +364,13 @@ def run_ours(args):
                          f"({len(records)} steps sampled)",
         "clocks": clk.summary(), "e2e": e2e, "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16, "kind": peak_kind},
     }
+    if rank == 0 and ws == 1 and not args.no_configs:
+        del path
+        torch.cuda.empty_cache()
+        try:
+            line["other_workloads"] = measure_configs(dev, hbm, int8_peak)
+        except Exception as exc:  # keep the main line; say what failed
+            line["other_workloads"] = {"error": f"{type(exc).__name__}: {exc}"}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(p, args.cpu_budget)
     if use_dist:
@@ -371,6 +378,156 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def _graph_time_us(torch, fns, reps):
+    """Mean device time of one call, the calls captured `reps` times round in one CUDA graph
+    (so launch overhead stays out) and the graph replayed once untimed, once timed."""
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for f in fns:
+            f()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for _ in range(reps):
+            for f in fns:
+                f()
+    with torch.cuda.stream(s):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        a.record()
+        g.replay()
+        b.record()
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) * 1e3 / (reps * len(fns))
+
+
+def measure_configs(dev, hbm, int8_peak):
+    """The other workloads, each timed alone after the main timed region (not part of the
+    step): the decode sweep (M in {1,4,16,64}, 4096 x 4096, eight weight copies rotated so the
+    weight streams from HBM), the LLM.int8 sweep (X [4096, 8192] with 0 / 8 / 82 outlier
+    columns, W [8192, 8192]), the 70B-shaped FFN GEMM (8192 x 28672 x 8192) and the variants
+    on X [8192, 8192] (two rotated copies, 268 MB > L2). Random device inputs of those shapes
+    and distributions; the parity tests cover the values."""
+    import torch
+
+    from w8a8_quantized_gemm_b200 import sq
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    out = {}
+
+    def hbm_entry(us, nbytes):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        return {"us": round(us, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
+
+    def tops_entry(us, ops):
+        t = ops / (us * 1e-6) / 1e12
+        return {"us": round(us, 2), "TOPS": round(t, 1), "frac_int8_peak": round(t / int8_peak, 4)}
+
+    # decode sweep: bytes N*K + M*K + 2*M*N + 4*(M+N) per call
+    N = K = 4096
+    Wqs = [torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev, generator=gen) for _ in range(8)]
+    e = torch.rand(N, device=dev, generator=gen) * 1e-3
+    dec = {}
+    for M in (1, 4, 16, 64):
+        Xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev, generator=gen)
+        d = torch.rand(M, device=dev, generator=gen) * 1e-2
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = sq.workspace(sq.SQ_OP_INT8_GEMM_DEQUANT, M, N, K, device=dev)
+        us = _graph_time_us(torch, [(lambda w=w: sq.sq_int8_gemm_dequant(Xq, w, d, e, sq.SQ_PER_CHANNEL, None, Y,
+                                                                         None, ws)) for w in Wqs], 10)
+        dec[f"M{M}"] = hbm_entry(us, N * K + M * K + 2 * M * N + 4 * (M + N))
+    out["decode_4096x4096"] = dec
+    del Wqs
+
+    # LLM.int8 sweep
+    M, N, K = 4096, 8192, 8192
+    base = (0.5 * torch.randn(M, K, device=dev, generator=gen)).clamp_(-5.5, 5.5)
+    W = (0.015 * torch.randn(N, K, device=dev, generator=gen)).to(torch.bfloat16)
+    Wq, ew = torch.empty((N, K), dtype=torch.int8, device=dev), torch.empty(N, device=dev)
+    sq.sq_smooth_quant_weight(W, None, sq.SQ_PER_CHANNEL, Wq, ew)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = sq.workspace(sq.SQ_OP_LLMINT8, M, N, K, device=dev)
+    cnt = torch.empty(1, dtype=torch.int32, device=dev)
+    llm = {}
+    for k_o in (0, 8, 82):
+        X = base.clone()
+        if k_o:
+            cols = torch.randperm(K, device=dev, generator=gen)[:k_o]
+            mag = 20.0 + 180.0 * torch.rand(k_o, device=dev, generator=gen)
+            X[:, cols] += mag * torch.where(torch.rand(k_o, device=dev, generator=gen) < 0.5, -1.0, 1.0)
+        X = X.to(torch.bfloat16)
+        us = _graph_time_us(torch, [lambda: sq.llmint8_decomposed_linear(X, W, Wq, ew, 6.0, None, Y, None, cnt, None,
+                                                                         ws)], 5)
+        found = int(cnt.item())
+        ent = tops_entry(us, 2.0 * M * N * K + 2.0 * M * N * found)
+        ent["k_outliers"] = found
+        llm[f"K_o={k_o}"] = ent
+    out["llmint8_4096x8192x8192"] = llm
+    del base, W, Wq, Y, ws, X
+
+    # 70B-shaped FFN GEMM with bias
+    M, N, K = 8192, 28672, 8192
+    Xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev, generator=gen)
+    Wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev, generator=gen)
+    d = torch.rand(M, device=dev, generator=gen) * 1e-2
+    e = torch.rand(N, device=dev, generator=gen) * 1e-3
+    bias = (0.1 * torch.randn(N, device=dev, generator=gen)).to(torch.bfloat16)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    us = _graph_time_us(torch, [lambda: sq.sq_int8_gemm_dequant(Xq, Wq, d, e, sq.SQ_PER_CHANNEL, bias, Y)], 3)
+    out["ffn70b_gemm_8192x28672x8192"] = tops_entry(us, 2.0 * M * N * K)
+    # the GEMM with asymmetric activations and with a per-tensor activation scale, same shape
+    z = torch.randint(-128, 128, (M,), dtype=torch.int32, device=dev, generator=gen)
+    rs = torch.empty(N, dtype=torch.int32, device=dev)
+    sq.sq_weight_row_sums(Wq, rs)
+    us = _graph_time_us(torch, [lambda: sq.sq_int8_gemm_dequant_ex(Xq, Wq, d, sq.SQ_PER_CHANNEL, z, e,
+                                                                   sq.SQ_PER_CHANNEL, rs, bias, Y)], 3)
+    out["gemm_asymmetric_8192x28672x8192"] = tops_entry(us, 2.0 * M * N * K)
+    us = _graph_time_us(torch, [lambda: sq.sq_int8_gemm_dequant_ex(Xq, Wq, d[:1], sq.SQ_PER_TENSOR, None, e,
+                                                                   sq.SQ_PER_CHANNEL, None, bias, Y)], 3)
+    out["gemm_per_tensor_x_8192x28672x8192"] = tops_entry(us, 2.0 * M * N * K)
+    us = _graph_time_us(torch, [lambda: sq.sq_weight_row_sums(Wq, rs)], 5)
+    out["weight_row_sums_28672x8192"] = hbm_entry(us, N * K + 4 * N)
+    del Xq, Wq, Y
+
+    # variants on X [8192, 8192]: algorithmic bytes read X once (+ write codes once)
+    M = K = 8192
+    Xs = [(1.5 * torch.randn(M, K, device=dev, generator=gen) + 0.2).to(torch.bfloat16) for _ in range(2)]
+    inv = torch.rand(K, device=dev, generator=gen) + 0.5
+    g = (torch.rand(K, device=dev, generator=gen) + 0.5).to(torch.bfloat16)
+    b = (0.1 * torch.randn(K, device=dev, generator=gen)).to(torch.bfloat16)
+    Xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    d, z = torch.empty(M, device=dev), torch.empty(M, dtype=torch.int32, device=dev)
+    d1, clip, thr = torch.empty(1, device=dev), torch.full((1,), 4.0, device=dev), torch.empty(1, device=dev)
+    wpt = sq.workspace(sq.SQ_OP_QUANT_ACT_PER_TENSOR, M, 0, K, device=dev)
+    wms = sq.workspace(sq.SQ_OP_MEAN_STD_THRESHOLD, M, 0, K, device=dev)
+    wpc = sq.workspace(sq.SQ_OP_ABS_PERCENTILE, M, 0, K, device=dev)
+    n = M * K
+    var = {}
+    cases = [
+        ("quant_act_per_token", 3 * n, lambda X: sq.sq_quant_act_per_token(X, inv, Xq, d)),
+        ("layernorm_smooth_quant", 3 * n, lambda X: sq.sq_norm_smooth_quant(X, sq.SQ_NORM_LAYER, g, b, 1e-5, inv, Xq,
+                                                                            d)),
+        ("rmsnorm_smooth_quant", 3 * n, lambda X: sq.sq_norm_smooth_quant(X, sq.SQ_NORM_RMS, g, None, 1e-5, inv, Xq,
+                                                                          d)),
+        ("quant_act_per_token_asym", 3 * n, lambda X: sq.sq_quant_act_per_token_asym(X, inv, Xq, d, z)),
+        ("quant_act_per_tensor_dynamic", 3 * n, lambda X: sq.sq_quant_act_per_tensor(X, inv, Xq, d1, None, wpt)),
+        ("quant_act_per_tensor_static_clip", 3 * n, lambda X: sq.sq_quant_act_per_tensor(X, inv, Xq, d1, clip)),
+        ("act_mean_std_threshold", 2 * n, lambda X: sq.sq_act_mean_std_threshold(X, 6.0, thr, None, wms)),
+        ("act_abs_percentile", 2 * n, lambda X: sq.sq_act_abs_percentile(X, 99.99, d1, wpc)),
+    ]
+    for name, nbytes, fn in cases:
+        us = _graph_time_us(torch, [(lambda X=X: fn(X)) for X in Xs], 5)
+        var[name] = hbm_entry(us, nbytes)
+    var["note"] = ("X bf16 [8192, 8192]; GB/s on the bytes of one read of X (+ one write of the int8 codes); the "
+                   "dynamic per-tensor form reads X twice by design (global maximum first)")
+    out["variants_8192x8192"] = var
+    sq.sq_sync_status()
+    return out
 
 
 def run_e2e(path, p, args, ops_step, use_dist, local, ws):
@@ -530,6 +687,7 @@ def main():
     ap.add_argument("--sample-every", type=int, default=10, help="timed steps per step carrying event nodes")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip timing the other workloads and the variants")
     ap.add_argument("--ref-rows", type=int, default=64, help="token rows per reference-arm step")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -257,7 +257,9 @@ SQ_API sq_status sq_int8_gemm_dequant_ex(const int8_t* Xq, const int8_t* Wq, con
  * Normalisation layer, smoothing and per-token quantization in one pass over X: the
  * smoothing folded into the output of the LayerNorm that precedes the linear layer
  * ([SQ] §4.2 fuse the scaling into the previous operation's output; §4.5 second detail).
- * Per row m, statistics summed in fp64 and rounded once to fp32:
+ * Per row m, statistics in fp64 rounded once to fp32 (computed in one pass from the sums of
+ * x and x^2; within fp64 rounding of the two-pass form below, so on rare rows a statistic
+ * may differ from a two-pass evaluation by one fp32 ulp):
  *   SQ_NORM_LAYER: mean = sum_k x / K, var = sum_k (x - mean)^2 / K,
  *                  rstd = fp32(1/sqrt(var + eps)), y = ((x - fp32(mean)) * rstd) * gamma_k + beta_k
  *   SQ_NORM_RMS:   rstd = fp32(1/sqrt(sum_k x^2 / K + eps)),   y = (x * rstd) * gamma_k + beta_k
@@ -274,8 +276,9 @@ SQ_API sq_status sq_norm_smooth_quant(const void* X_bf16, int64_t M, int64_t K, 
  * Data-dependent outlier threshold: threshold = mean + k * std over all M*K elements of X,
  * std the unbiased standard deviation. [LLMINT8] §3.1 pre-screening (threshold = mu + 6
  * sigma from the layer's activation statistics); [QAT] §2.1 (mean + 3 std).
- * mean and the sum of squared deviations are summed in fp64 (two passes over X, fixed
- * summation order: the result is deterministic); the threshold is rounded once to fp32.
+ * One pass over X: the sums of x and x^2 in fp64 (fixed summation order, so the result is
+ * deterministic), mean = S1/n, var = (S2 - S1*mean)/(n-1); the threshold is rounded once
+ * to fp32.
  * threshold: fp32 [1] device. mean_std: fp64 [2] device (mean, std) or NULL.
  * ws: sq_workspace_size(SQ_OP_MEAN_STD_THRESHOLD, M, 0, K) bytes.
  */

@@ -96,8 +96,8 @@ def test_llmint8_validation():
 
 def test_variant_workspace_sizes():
     assert sq.sq_workspace_size(sq.SQ_OP_QUANT_ACT_PER_TENSOR, 16, 0, 64) >= 4
-    assert sq.sq_workspace_size(sq.SQ_OP_MEAN_STD_THRESHOLD, 4096, 0, 8192) >= 8 * (2 * 1024 + 2)
-    assert sq.sq_workspace_size(sq.SQ_OP_MEAN_STD_THRESHOLD, 3, 0, 64) >= 8 * (2 * 3 + 2)
+    assert sq.sq_workspace_size(sq.SQ_OP_MEAN_STD_THRESHOLD, 4096, 0, 8192) >= 8 * 2 * 1024
+    assert sq.sq_workspace_size(sq.SQ_OP_MEAN_STD_THRESHOLD, 3, 0, 64) >= 8 * 2 * 3
     assert sq.sq_workspace_size(sq.SQ_OP_ABS_PERCENTILE, 1, 0, 16) == 8 * (1 << 15)
 
 

@@ -100,5 +100,32 @@ __device__ __forceinline__ double group_sum(double a, double* red /* [CTA thread
   return a;
 }
 
+// Two fp64 sums over the TPR threads of one row group at once (one shared-memory round).
+template <int TPR>
+__device__ __forceinline__ void group_sum2(double& a, double& b, double2* red /* [CTA threads / 32] */) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a = __dadd_rn(a, __shfl_xor_sync(0xffffffffu, a, o));
+    b = __dadd_rn(b, __shfl_xor_sync(0xffffffffu, b, o));
+  }
+  if constexpr (TPR > 32) {
+    constexpr int kWarpsPerGroup = TPR / 32;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g0 = (warp / kWarpsPerGroup) * kWarpsPerGroup;
+    if (lane == 0) red[warp] = make_double2(a, b);
+    __syncthreads();
+    double2 t = red[g0];
+#pragma unroll
+    for (int w = 1; w < kWarpsPerGroup; ++w) {
+      t.x = __dadd_rn(t.x, red[g0 + w].x);
+      t.y = __dadd_rn(t.y, red[g0 + w].y);
+    }
+    __syncthreads();
+    a = t.x;
+    b = t.y;
+  }
+}
+
 }  // namespace rows
 }  // namespace sq

@@ -94,7 +94,7 @@ norm_quant_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
   griddep_wait();
   griddep_launch_dependents();
   __shared__ float redf[kThreads / 32];
-  __shared__ double redd[kThreads / 32];
+  __shared__ double2 redd[kThreads / 32];
   const int g = threadIdx.x / TPR;
   const int t = threadIdx.x % TPR;
   const int64_t step = static_cast<int64_t>(TPR) * 16;
@@ -169,37 +169,32 @@ norm_quant_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
         if (k < K) raw16(src + nrow * ld + k, raw[c]);
       }
     }
-    // row statistics in fp64 (absent columns hold 0 and are skipped in the deviations)
-    float mean_f = 0.0f;
-    double ss = 0.0;
-    if (layer) {
-      double s1 = 0.0;
+    // row statistics in one pass: sum and sum of squares in fp64 (the square of a bf16
+    // value is exact in fp64), four independent chains per thread, one group reduction;
+    // var = E[x^2] - mean^2 (the fp64 headroom keeps it within rounding of the two-pass form
+    // for any input a bf16 row can hold relative to fp32 resolution). Absent columns hold 0.
+    double s1a = 0.0, s1b = 0.0, s2a = 0.0, s2b = 0.0;
 #pragma unroll
-      for (int c = 0; c < CHUNKS; ++c)
+    for (int c = 0; c < CHUNKS; ++c)
 #pragma unroll
-        for (int i = 0; i < 16; ++i) s1 = __dadd_rn(s1, static_cast<double>(x[c][i]));
-      const double mean = __ddiv_rn(group_sum<TPR>(s1, redd), static_cast<double>(K));
-      mean_f = __double2float_rn(mean);
-#pragma unroll
-      for (int c = 0; c < CHUNKS; ++c) {
-        if (c * step + t * 16 < K) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const double dv = __dsub_rn(static_cast<double>(x[c][i]), mean);
-            ss = __dadd_rn(ss, __dmul_rn(dv, dv));
-          }
-        }
+      for (int i = 0; i < 16; i += 2) {
+        const double xa = static_cast<double>(x[c][i]);
+        const double xb = static_cast<double>(x[c][i + 1]);
+        s1a = __dadd_rn(s1a, xa);
+        s1b = __dadd_rn(s1b, xb);
+        s2a = __fma_rn(xa, xa, s2a);
+        s2b = __fma_rn(xb, xb, s2b);
       }
-    } else {
-#pragma unroll
-      for (int c = 0; c < CHUNKS; ++c)
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const double dv = static_cast<double>(x[c][i]);
-          ss = __dadd_rn(ss, __dmul_rn(dv, dv));
-        }
+    double s1 = __dadd_rn(s1a, s1b), s2 = __dadd_rn(s2a, s2b);
+    group_sum2<TPR>(s1, s2, redd);
+    const double kd = static_cast<double>(K);
+    float mean_f = 0.0f;
+    double m2 = __ddiv_rn(s2, kd);
+    if (layer) {
+      const double mean = __ddiv_rn(s1, kd);
+      mean_f = __double2float_rn(mean);
+      m2 = fmax(__dsub_rn(m2, __dmul_rn(mean, mean)), 0.0);
     }
-    const double m2 = __ddiv_rn(group_sum<TPR>(ss, redd), static_cast<double>(K));
     const float rstd_f = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(m2, static_cast<double>(eps)))));
     // y = ((x - mean) * rstd) * gamma + beta, x' = y * inv_s, absmax
     float a = 0.0f;
@@ -258,20 +253,18 @@ cudaError_t launch_norm_t(const uint16_t* src, int64_t rows, int64_t K, int64_t 
 // ------------------------------------------------------------------ mean / std threshold
 constexpr int kStatThreads = 256;
 
-// partial[b] = sum of the elements of CTA b's rows (fp64, fixed order).
+// part1[b], part2[b] = sum and sum of squares of the elements of CTA b's rows (fp64, four
+// independent chains per thread, then a fixed-order CTA reduction).
 __global__ void __launch_bounds__(kStatThreads)
 sum_partials_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int64_t rows_per_cta,
-                    const double* __restrict__ mean_in, double* __restrict__ partial) {
+                    double* __restrict__ part1, double* __restrict__ part2) {
   griddep_wait();
   griddep_launch_dependents();
-  __shared__ double red[kStatThreads / 32];
-  // second pass: sum of squared deviations from the mean of the first
-  const bool dev = mean_in != nullptr;
-  const double mean = dev ? *mean_in : 0.0;
+  __shared__ double2 red[kStatThreads / 32];
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows_per_cta;
   const int64_t r1 = min(rows, r0 + rows_per_cta);
   const int64_t vecs = K / 8;
-  double acc = 0.0;
+  double s1a = 0.0, s1b = 0.0, s2a = 0.0, s2b = 0.0;
   for (int64_t r = r0; r < r1; ++r) {
     const uint4* p = reinterpret_cast<const uint4*>(src + r * ld);
     for (int64_t v = threadIdx.x; v < vecs; v += kStatThreads) {
@@ -281,45 +274,44 @@ sum_partials_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, i
       for (int i = 0; i < 4; ++i) {
         const double lo = static_cast<double>(__uint_as_float(u[i] << 16));
         const double hi = static_cast<double>(__uint_as_float(u[i] & 0xFFFF0000u));
-        if (dev) {
-          const double a = __dsub_rn(lo, mean), b = __dsub_rn(hi, mean);
-          acc = __dadd_rn(acc, __dmul_rn(a, a));
-          acc = __dadd_rn(acc, __dmul_rn(b, b));
-        } else {
-          acc = __dadd_rn(acc, lo);
-          acc = __dadd_rn(acc, hi);
-        }
+        s1a = __dadd_rn(s1a, lo);
+        s1b = __dadd_rn(s1b, hi);
+        s2a = __fma_rn(lo, lo, s2a);
+        s2b = __fma_rn(hi, hi, s2b);
       }
     }
   }
-  acc = group_sum<kStatThreads>(acc, red);
-  if (threadIdx.x == 0) partial[blockIdx.x] = acc;
+  double s1 = __dadd_rn(s1a, s1b), s2 = __dadd_rn(s2a, s2b);
+  group_sum2<kStatThreads>(s1, s2, red);
+  if (threadIdx.x == 0) {
+    part1[blockIdx.x] = s1;
+    part2[blockIdx.x] = s2;
+  }
 }
 
-// One CTA: total = sum of the G partials in a fixed order; writes total / divisor to *out.
+// One CTA: totals of the G partials in a fixed order, mean = S1/n, unbiased
+// var = (S2 - S1*mean)/(n - 1), threshold = fp32(mean + k*sqrt(var)).
 __global__ void __launch_bounds__(kStatThreads)
-reduce_partials_kernel(const double* __restrict__ partial, int G, double divisor, double* __restrict__ out) {
+finish_threshold_kernel(const double* __restrict__ part1, const double* __restrict__ part2, int G, double n,
+                        double k, float* __restrict__ threshold, double* __restrict__ mean_std) {
   griddep_wait();
   griddep_launch_dependents();
-  __shared__ double red[kStatThreads / 32];
-  double acc = 0.0;
-  for (int i = threadIdx.x; i < G; i += kStatThreads) acc = __dadd_rn(acc, partial[i]);
-  acc = group_sum<kStatThreads>(acc, red);
-  if (threadIdx.x == 0) *out = __ddiv_rn(acc, divisor);
-}
-
-// threshold = fp32(mean + k * sqrt(var)), var = ss / (n - 1) already in stats[1].
-__global__ void threshold_kernel(const double* __restrict__ stats, double k, float* __restrict__ threshold,
-                                 double* __restrict__ mean_std) {
-  griddep_wait();
-  griddep_launch_dependents();
-  if (threadIdx.x != 0) return;
-  const double mean = stats[0];
-  const double sd = __dsqrt_rn(stats[1]);
-  *threshold = __double2float_rn(__dadd_rn(mean, __dmul_rn(k, sd)));
-  if (mean_std != nullptr) {
-    mean_std[0] = mean;
-    mean_std[1] = sd;
+  __shared__ double2 red[kStatThreads / 32];
+  double s1 = 0.0, s2 = 0.0;
+  for (int i = threadIdx.x; i < G; i += kStatThreads) {
+    s1 = __dadd_rn(s1, part1[i]);
+    s2 = __dadd_rn(s2, part2[i]);
+  }
+  group_sum2<kStatThreads>(s1, s2, red);
+  if (threadIdx.x == 0) {
+    const double mean = __ddiv_rn(s1, n);
+    const double var = n > 1.0 ? fmax(__ddiv_rn(__dsub_rn(s2, __dmul_rn(s1, mean)), n - 1.0), 0.0) : 0.0;
+    const double sd = __dsqrt_rn(var);
+    *threshold = __double2float_rn(__dadd_rn(mean, __dmul_rn(k, sd)));
+    if (mean_std != nullptr) {
+      mean_std[0] = mean;
+      mean_std[1] = sd;
+    }
   }
 }
 
@@ -417,8 +409,8 @@ cudaError_t launch_norm_quant(const uint16_t* src, int64_t rows, int64_t K, int6
 int64_t mean_std_ctas(int64_t rows) { return std::min<int64_t>(rows, 1024); }
 
 size_t mean_std_workspace_bytes(int64_t rows) {
-  // two partial arrays of G doubles and two statistics
-  return sizeof(double) * (2 * static_cast<size_t>(mean_std_ctas(rows)) + 2);
+  // the two partial arrays of G doubles
+  return sizeof(double) * 2 * static_cast<size_t>(mean_std_ctas(rows));
 }
 
 cudaError_t launch_mean_std_threshold(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, double k,
@@ -428,23 +420,13 @@ cudaError_t launch_mean_std_threshold(const uint16_t* src, int64_t rows, int64_t
   const int64_t ctas = (rows + rpc - 1) / rpc;
   double* part1 = static_cast<double*>(ws);
   double* part2 = part1 + G;
-  double* stats = part2 + G;  // [0] mean, [1] variance
   const double n = static_cast<double>(rows) * static_cast<double>(K);
   cudaError_t e = launch_kernel(sum_partials_kernel, dim3(static_cast<unsigned>(ctas)), dim3(kStatThreads), 0,
-                                stream, false, src, rows, K, ld, rpc, static_cast<const double*>(nullptr), part1);
+                                stream, false, src, rows, K, ld, rpc, part1, part2);
   if (e == cudaSuccess)
-    e = launch_kernel(reduce_partials_kernel, dim3(1), dim3(kStatThreads), 0, stream, false,
-                      static_cast<const double*>(part1), static_cast<int>(ctas), n, stats);
-  if (e == cudaSuccess)
-    e = launch_kernel(sum_partials_kernel, dim3(static_cast<unsigned>(ctas)), dim3(kStatThreads), 0, stream, false,
-                      src, rows, K, ld, rpc, static_cast<const double*>(stats), part2);
-  if (e == cudaSuccess)
-    e = launch_kernel(reduce_partials_kernel, dim3(1), dim3(kStatThreads), 0, stream, false,
-                      static_cast<const double*>(part2), static_cast<int>(ctas), n > 1.0 ? n - 1.0 : 1.0,
-                      stats + 1);
-  if (e == cudaSuccess)
-    e = launch_kernel(threshold_kernel, dim3(1), dim3(32), 0, stream, false, static_cast<const double*>(stats), k,
-                      threshold, mean_std);
+    e = launch_kernel(finish_threshold_kernel, dim3(1), dim3(kStatThreads), 0, stream, false,
+                      static_cast<const double*>(part1), static_cast<const double*>(part2), static_cast<int>(ctas), n,
+                      k, threshold, mean_std);
   return e;
 }
 

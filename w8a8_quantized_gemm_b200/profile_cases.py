@@ -1,6 +1,7 @@
 """Small, self-contained launches of single kernels for profiler captures (ncu).
 
-Usage: python -m w8a8_quantized_gemm_b200.profile_cases {gemm,decode,llm,quant,absmax}
+Usage: python -m w8a8_quantized_gemm_b200.profile_cases
+       {gemm,decode,llm,quant,absmax,norm,asym,meanstd,percentile,rowsums,gemm_asym}
 
 Each case makes random device inputs of one workload's shape and calls one entry point three
 times (so that a capture can skip the first, cold launch):
@@ -9,6 +10,12 @@ times (so that a capture can skip the first, cold launch):
   llm     llmint8_decomposed_linear, 2048 x 11008 x 4096 with 4 outlier columns
   quant   sq_quant_act_per_token with smoothing, X bf16 [8192, 8192] (inputs larger than L2)
   absmax  sq_act_channel_absmax, X bf16 [8192, 8192]
+  norm    sq_norm_smooth_quant (LayerNorm with beta, smoothing), X bf16 [8192, 8192]
+  asym    sq_quant_act_per_token_asym with smoothing, X bf16 [8192, 8192]
+  meanstd sq_act_mean_std_threshold (k = 6), X bf16 [8192, 8192]
+  percentile  sq_act_abs_percentile (99.99), X bf16 [8192, 8192]
+  rowsums sq_weight_row_sums, Wq int8 [28672, 8192]
+  gemm_asym  sq_int8_gemm_dequant_ex with asymmetric activations, 2048 x 11008 x 4096
 """
 import sys
 
@@ -57,6 +64,43 @@ def main(mode: str) -> None:
             amax = torch.empty(K, device=dev)
             for _ in range(3):
                 sq.sq_act_channel_absmax(X, amax)
+    elif mode in ("norm", "asym", "meanstd", "percentile"):
+        M, K = 8192, 8192
+        X = (torch.randn(M, K, device=dev) * 1.5 + 0.2).to(torch.bfloat16)
+        Xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        dd = torch.empty(M, device=dev)
+        inv = torch.rand(K, device=dev) + 0.5
+        for _ in range(3):
+            if mode == "norm":
+                g = (torch.rand(K, device=dev) + 0.5).to(torch.bfloat16)
+                b = (torch.randn(K, device=dev) * 0.1).to(torch.bfloat16)
+                sq.sq_norm_smooth_quant(X, sq.SQ_NORM_LAYER, g, b, 1e-5, inv, Xq, dd)
+            elif mode == "asym":
+                z = torch.empty(M, dtype=torch.int32, device=dev)
+                sq.sq_quant_act_per_token_asym(X, inv, Xq, dd, z)
+            elif mode == "meanstd":
+                thr = torch.empty(1, device=dev)
+                sq.sq_act_mean_std_threshold(X, 6.0, thr, None, sq.workspace(sq.SQ_OP_MEAN_STD_THRESHOLD, M, 0, K))
+            else:
+                out = torch.empty(1, device=dev)
+                sq.sq_act_abs_percentile(X, 99.99, out, sq.workspace(sq.SQ_OP_ABS_PERCENTILE, M, 0, K))
+    elif mode == "rowsums":
+        Wq = torch.randint(-127, 128, (28672, 8192), dtype=torch.int8, device=dev)
+        rs = torch.empty(28672, dtype=torch.int32, device=dev)
+        for _ in range(3):
+            sq.sq_weight_row_sums(Wq, rs)
+    elif mode == "gemm_asym":
+        M, N, K = 2048, 11008, 4096
+        Xq = torch.randint(-128, 128, (M, K), dtype=torch.int8, device=dev)
+        Wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev)
+        d = torch.rand(M, device=dev) * 1e-2
+        e = torch.rand(N, device=dev) * 1e-3
+        z = torch.randint(-128, 128, (M,), dtype=torch.int32, device=dev)
+        rs = torch.empty(N, dtype=torch.int32, device=dev)
+        sq.sq_weight_row_sums(Wq, rs)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            sq.sq_int8_gemm_dequant_ex(Xq, Wq, d, sq.SQ_PER_CHANNEL, z, e, sq.SQ_PER_CHANNEL, rs, None, Y)
     else:
         raise SystemExit(f"unknown case {mode!r}")
     sq.sq_sync_status()

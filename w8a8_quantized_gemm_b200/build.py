@@ -21,7 +21,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsq.so")
 
 SOURCES = ["sq_api.cu", "sq_reduce.cu", "sq_quant.cu", "sq_outlier.cu", "sq_gemm.cu", "sq_noalloc.cu",
-           "sq_variants.cu"]
+           "sq_variants.cu", "sq_gemv.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
               "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

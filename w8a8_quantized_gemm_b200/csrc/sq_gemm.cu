@@ -9,14 +9,17 @@
 // "LLM.int8()技术解析：8位量化如何优化大语言模型计算" §3.1 (normal columns in an INT8 GEMM,
 //   outlier columns in a 16-bit GEMM, results merged).
 //
-// Structure (one persistent CTA per SM, 6 warps):
+// Up to 4 tokens (no outlier product) take the CUDA-core product of sq_gemv.cu instead.
+//
+// Structure (one persistent CTA per SM, 10 warps):
 //   warp 0     TMA producer: 128x128-byte A tiles and BNx128-byte B tiles into a ring of
 //              shared-memory stages (128-byte swizzle), completion on `full` mbarriers;
 //   warp 1     allocates TMEM; one lane issues tcgen05.mma (4 x K=32 bytes per stage) into
 //              a double-buffered accumulator and frees stages with tcgen05.commit;
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one output row per
-//              thread), y = (float(acc) * d_m) * e_n (+ o) (+ bias) -> bf16, global stores;
-//              overlaps the next tile's main loop through the second TMEM buffer.
+//   warps 2-9  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one output row per
+//              thread, two column halves), y = (float(acc) * d_m) * e_n (+ o) (+ bias) -> bf16,
+//              TMA stores through shared-memory staging; overlaps the next tile's main loop
+//              through the second TMEM buffer.
 // For a few tokens (M <= 64) the operands swap roles: the weight supplies the 128-row MMA
 // operand (output channels on TMEM lanes) and the tokens the N dimension, so no MMA row
 // and no weight byte is spent on padding; the epilogue then applies the per-token scale
@@ -820,6 +823,7 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
 }  // namespace
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, bool outliers) {
+  if (gemv_applies(M, K, outliers)) return 0;
   const Plan pl = plan_gemm(M, N, K, outliers);
   if (pl.tail_tiles == 0) return 0;
   return up256(sizeof(int32_t) * pl.tail_tiles * pl.splits * kBM * pl.bn) +
@@ -828,6 +832,8 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, bool outliers) {
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream, const char** why) {
   const bool outliers = a.Xo != nullptr;
+  // up to 4 tokens: a weight stream on the CUDA cores (no tensor-core set-up, no K split)
+  if (gemv_applies(a.M, a.K, outliers) && a.fault == 0) return launch_gemv(a, stream);
   const Plan pl = plan_gemm(a.M, a.N, a.K, outliers);
   if (outliers) {
     // int32 + fp32 accumulators: 256-wide tiles fit TMEM once, narrower ones twice

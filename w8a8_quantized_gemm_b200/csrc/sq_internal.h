@@ -148,4 +148,8 @@ struct GemmArgs {
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, bool outliers);
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream, const char** why);
 
+// ---- CUDA-core product for M <= 4 tokens (sq_gemv.cu): same arguments and results as the GEMM.
+bool gemv_applies(int64_t M, int64_t K, bool outliers);
+cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t stream);
+
 }  // namespace sq

@@ -1,12 +1,13 @@
 """Small, self-contained launches of single kernels for profiler captures (ncu).
 
 Usage: python -m w8a8_quantized_gemm_b200.profile_cases
-       {gemm,decode,llm,quant,absmax,norm,asym,meanstd,percentile,rowsums,gemm_asym}
+       {gemm,decode,decode1,llm,quant,absmax,norm,asym,meanstd,percentile,rowsums,gemm_asym}
 
 Each case makes random device inputs of one workload's shape and calls one entry point three
 times (so that a capture can skip the first, cold launch):
   gemm    sq_int8_gemm_dequant, 2048 x 11008 x 4096 (Llama-2-7B MLP up-projection)
-  decode  sq_int8_gemm_dequant, 64 x 4096 x 4096 (decode, split K)
+  decode  sq_int8_gemm_dequant, 64 x 4096 x 4096 (decode: swapped operands, split K)
+  decode1 sq_int8_gemm_dequant, 1 x 4096 x 4096 (one token: the CUDA-core product)
   llm     llmint8_decomposed_linear, 2048 x 11008 x 4096 with 4 outlier columns
   quant   sq_quant_act_per_token with smoothing, X bf16 [8192, 8192] (inputs larger than L2)
   absmax  sq_act_channel_absmax, X bf16 [8192, 8192]
@@ -28,8 +29,8 @@ def main(mode: str) -> None:
     torch.cuda.set_device(0)
     dev = "cuda"
     torch.manual_seed(0)
-    if mode in ("gemm", "decode"):
-        M, N, K = (2048, 11008, 4096) if mode == "gemm" else (64, 4096, 4096)
+    if mode in ("gemm", "decode", "decode1"):
+        M, N, K = {"gemm": (2048, 11008, 4096), "decode": (64, 4096, 4096), "decode1": (1, 4096, 4096)}[mode]
         Xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev)
         Wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev)
         d = torch.rand(M, device=dev) * 1e-2

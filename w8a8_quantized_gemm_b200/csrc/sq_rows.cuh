@@ -14,9 +14,13 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
          ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
 }
 
+// clamp(rne(x * r), -128, 127), returned in the low byte (the upper bytes are not the code).
+// The product is clamped first (the same result: every value in [127, 128) rounds to 127 or
+// 128 and clamps to 127, likewise at -128), then rounded half to even by adding 1.5 * 2^23,
+// whose fp32 sum keeps the integer in its low mantissa bits: no float->int conversion unit.
 __device__ __forceinline__ int q8(float x, float r) {
-  int q = __float2int_rn(__fmul_rn(x, r));
-  return min(127, max(-128, q));
+  const float t = fminf(fmaxf(__fmul_rn(x, r), -128.0f), 127.0f);
+  return __float_as_int(__fadd_rn(t, 12582912.0f));
 }
 
 __device__ __forceinline__ void store_q16(int8_t* dst, const float (&v)[16], float r) {

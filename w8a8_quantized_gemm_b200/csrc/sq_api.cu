@@ -305,9 +305,13 @@ sq_status llm_impl(const char* fn, const void* X_bf16, const void* W_bf16, const
     ov.count = count;
     ov.gathered = Xo;
     ov.ld_gathered = L.ldo;
+    ov.w_src = W;
+    ov.w_rows = N;
+    ov.w_ld = K;
+    ov.idx = idx;
+    ov.w_gathered = Wo;
     e = sq::launch_quant_rows(X, M, K, K, nullptr, ov, Xq, d, cs);
   }
-  if (e == cudaSuccess) e = sq::launch_gather_columns(W, N, K, idx, count, Wo, L.ldo, cs);
   if (e != cudaSuccess) return cuda_fail(e, fn);
   sq::GemmArgs a;
   a.Xq = Xq;

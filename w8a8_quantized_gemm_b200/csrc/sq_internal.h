@@ -79,6 +79,11 @@ struct OutlierView {
   const int32_t* count = nullptr;    // [1] number of outliers
   uint16_t* gathered = nullptr;      // [rows, ld_gathered] bf16 outlier values (zero padded to 64)
   int64_t ld_gathered = 0;
+  // the same kernel also gathers the weight's outlier columns (one thread per weight row):
+  const uint16_t* w_src = nullptr;   // [w_rows, w_ld] bf16, or nullptr
+  int64_t w_rows = 0, w_ld = 0;
+  const int32_t* idx = nullptr;      // [count] ascending outlier column indices
+  uint16_t* w_gathered = nullptr;    // [w_rows, ld_gathered]
 };
 
 // Per-row smooth + quantize: q[r,k] = clamp(rne(src[r,k]*vec[k] * 127/a_r)), scale[r] = a_r/127.
@@ -99,9 +104,6 @@ cudaError_t launch_quant_rows_asym(const uint16_t* src, int64_t rows, int64_t K,
 cudaError_t launch_outlier_mask(const float* amax, int64_t K, float threshold, const float* threshold_dev,
                                 uint32_t* mask, int32_t* prefix, int32_t* idx, int32_t* count, uint32_t* mask_out,
                                 int32_t* count_out, cudaStream_t stream);
-// dst[r, c] = c < count ? src[r, idx[c]] : 0 for c < roundup(count, 64).
-cudaError_t launch_gather_columns(const uint16_t* src, int64_t rows, int64_t ld, const int32_t* idx,
-                                  const int32_t* count, uint16_t* dst, int64_t ld_dst, cudaStream_t stream);
 
 // ---- variants (sq_variants.cu)
 // s <- max(s / max(s) * 127, 1e-5), inv_s = 1/s (one CTA).

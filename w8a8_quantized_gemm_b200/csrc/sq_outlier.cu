@@ -1,5 +1,5 @@
-// LLM.int8() outlier-column bookkeeping: bitmask, ascending index list, per-word
-// prefix counts, and the gather of outlier columns into a dense bf16 operand.
+// LLM.int8() outlier-column bookkeeping: bitmask, ascending index list and per-word prefix
+// counts (the gathers of the outlier columns run inside the masked row quantization).
 //
 // "LLM.int8()技术解析：8位量化如何优化大语言模型计算" §2.1 (a column whose absmax exceeds the
 // threshold is an outlier column) and §3.1 (real-time detection marks outlier
@@ -12,98 +12,105 @@ namespace sq {
 namespace {
 
 constexpr int kMaskThreads = 1024;
+constexpr int kMaskWarps = kMaskThreads / 32;
+constexpr int kMaxWords = 65536 / 32;  // K <= 65536
 
-// One CTA. Column j is handled by thread j % 1024 of pass j / 1024: a warp covers one
-// 32-column mask word, so the ballot is the word and the scan runs over warps. The flags of
-// the first kPrefetch passes are computed from loads issued before the scan loop (one memory
-// round trip for K <= 8192).
-constexpr int kPrefetch = 8;
-
+// One CTA. Warp w owns the mask words [w*wpw, (w+1)*wpw), wpw = ceil(words/32); in batch b
+// lane l handles word w*wpw + 32b + l and reads its 32 column maxima (128 contiguous bytes).
+// Pass 1 forms the words (kept in shared memory) and each warp's outlier count; one scan
+// over the 32 warp counts gives each warp's base; pass 2 scans the words' popcounts within
+// the warp, batch by batch, and writes each word, its prefix and the ascending index list.
+// Two block-wide barriers in all, whatever K.
 __global__ void __launch_bounds__(kMaskThreads)
 outlier_mask_kernel(const float* __restrict__ amax, int64_t K, float threshold_value,
                     const float* __restrict__ threshold_dev, uint32_t* __restrict__ mask,
                     int32_t* __restrict__ prefix, int32_t* __restrict__ idx, int32_t* __restrict__ count,
                     uint32_t* __restrict__ mask_out, int32_t* __restrict__ count_out) {
-  __shared__ int32_t warp_cnt[kMaskThreads / 32];
-  __shared__ int32_t warp_off[kMaskThreads / 32];
-  __shared__ int32_t running;
+  __shared__ uint32_t words_s[kMaxWords];
+  __shared__ int32_t warp_base[kMaskWarps + 1];
   griddep_wait();
   griddep_launch_dependents();
   const float threshold = threshold_dev != nullptr ? __ldg(threshold_dev) : threshold_value;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int64_t words = (K + 31) / 32;
-  bool pre[kPrefetch];
+  const int64_t wpw = (words + kMaskWarps - 1) / kMaskWarps;
+  const int64_t w_begin = warp * wpw;
+  const int64_t w_end = w_begin + wpw < words ? w_begin + wpw : words;
+
+  // pass 1: the words and this warp's count
+  int32_t warp_total = 0;
+  for (int64_t b0 = w_begin; b0 < w_end; b0 += 32) {
+    const int64_t word = b0 + lane;
+    uint32_t bits = 0u;
+    if (word < w_end) {
+      const int64_t j0 = word * 32;
+      if (j0 + 32 <= K) {
+        const float4* p = reinterpret_cast<const float4*>(amax + j0);
 #pragma unroll
-  for (int i = 0; i < kPrefetch; ++i) {
-    const int64_t j = static_cast<int64_t>(i) * kMaskThreads + threadIdx.x;
-    pre[i] = (j < K) && (__ldg(amax + j) > threshold);
-  }
-  if (threadIdx.x == 0) running = 0;
-  __syncthreads();
-  int pass = 0;
-  for (int64_t base = 0; base < K; base += kMaskThreads, ++pass) {
-    const int64_t j = base + threadIdx.x;
-    bool flag = false;
-#pragma unroll
-    for (int i = 0; i < kPrefetch; ++i)
-      if (i == pass) flag = pre[i];
-    if (pass >= kPrefetch) flag = (j < K) && (__ldg(amax + j) > threshold);
-    const uint32_t ballot = __ballot_sync(0xffffffffu, flag);
-    if (lane == 0) warp_cnt[warp] = __popc(ballot);
-    __syncthreads();
-    if (warp == 0) {
-      const int32_t c = warp_cnt[lane];
-      int32_t incl = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+        for (int q = 0; q < 8; ++q) {
+          const float4 v = __ldg(p + q);
+          bits |= (v.x > threshold ? 1u : 0u) << (4 * q);
+          bits |= (v.y > threshold ? 1u : 0u) << (4 * q + 1);
+          bits |= (v.z > threshold ? 1u : 0u) << (4 * q + 2);
+          bits |= (v.w > threshold ? 1u : 0u) << (4 * q + 3);
+        }
+      } else {
+        for (int i = 0; i < 32 && j0 + i < K; ++i) bits |= (__ldg(amax + j0 + i) > threshold ? 1u : 0u) << i;
       }
-      warp_off[lane] = running + incl - c;
+      words_s[word] = bits;
     }
-    __syncthreads();
-    const int64_t word = (base >> 5) + warp;
-    if (lane == 0 && word < words) {
-      mask[word] = ballot;
-      prefix[word] = warp_off[warp];
-      if (mask_out) mask_out[word] = ballot;
+    int32_t c = __popc(bits);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    warp_total += c;
+  }
+  if (lane == 0) warp_base[warp] = warp_total;
+  __syncthreads();
+  if (warp == 0) {
+    const int32_t c = warp_base[lane];
+    int32_t incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
-    if (flag) idx[warp_off[warp] + __popc(ballot & ((1u << lane) - 1u))] = static_cast<int32_t>(j);
-    __syncthreads();
-    if (threadIdx.x == kMaskThreads - 1) running = warp_off[warp] + __popc(ballot);
-    __syncthreads();
+    __syncwarp();
+    warp_base[lane] = incl - c;
+    if (lane == 31) warp_base[kMaskWarps] = incl;
+  }
+  __syncthreads();
+
+  // pass 2: prefixes and the index list
+  int32_t running = warp_base[warp];
+  for (int64_t b0 = w_begin; b0 < w_end; b0 += 32) {
+    const int64_t word = b0 + lane;
+    const uint32_t bits = word < w_end ? words_s[word] : 0u;
+    const int32_t c = __popc(bits);
+    int32_t incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int32_t excl = running + incl - c;
+    if (word < w_end) {
+      mask[word] = bits;
+      prefix[word] = excl;
+      if (mask_out) mask_out[word] = bits;
+      uint32_t rest = bits;
+      int32_t pos = excl;
+      while (rest) {
+        const int i = __ffs(rest) - 1;
+        idx[pos++] = static_cast<int32_t>(word * 32 + i);
+        rest &= rest - 1u;
+      }
+    }
+    running += __shfl_sync(0xffffffffu, incl, 31);
   }
   if (threadIdx.x == 0) {
-    count[0] = running;
-    if (count_out) count_out[0] = running;
-  }
-}
-
-// One thread per row: dst[r, c] = src[r, idx[c]] for c < count, 0 for count <= c <
-// roundup(count, 64), written 8 columns (16 bytes) at a time.
-__global__ void gather_columns_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t ld,
-                                      const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
-                                      uint16_t* __restrict__ dst, int64_t ld_dst) {
-  griddep_wait();
-  griddep_launch_dependents();
-  const int32_t cnt = __ldg(count);
-  const int32_t padded = (cnt + 63) & ~63;
-  for (int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; r < rows;
-       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const uint16_t* srow = src + r * ld;
-    uint4* drow = reinterpret_cast<uint4*>(dst + r * ld_dst);
-    for (int32_t c0 = 0; c0 < padded; c0 += 8) {
-      uint32_t w[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int32_t c = c0 + 2 * i;
-        const uint32_t lo = c < cnt ? srow[__ldg(idx + c)] : 0u;
-        const uint32_t hi = c + 1 < cnt ? srow[__ldg(idx + c + 1)] : 0u;
-        w[i] = lo | (hi << 16);
-      }
-      drow[c0 / 8] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
+    count[0] = warp_base[kMaskWarps];
+    if (count_out) count_out[0] = warp_base[kMaskWarps];
   }
 }
 
@@ -114,16 +121,6 @@ cudaError_t launch_outlier_mask(const float* amax, int64_t K, float threshold, c
                                 int32_t* count_out, cudaStream_t stream) {
   return launch_kernel(outlier_mask_kernel, dim3(1), dim3(kMaskThreads), 0, stream, false, amax, K, threshold,
                        threshold_dev, mask, prefix, idx, count, mask_out, count_out);
-}
-
-cudaError_t launch_gather_columns(const uint16_t* src, int64_t rows, int64_t ld, const int32_t* idx,
-                                  const int32_t* count, uint16_t* dst, int64_t ld_dst, cudaStream_t stream) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t blocks = std::min<int64_t>((rows + 127) / 128, static_cast<int64_t>(sms) * 8);
-  return launch_kernel(gather_columns_kernel, dim3(static_cast<unsigned>(blocks)), dim3(128), 0, stream, false,
-                       src, rows, ld, idx, count, dst, ld_dst);
 }
 
 }  // namespace sq

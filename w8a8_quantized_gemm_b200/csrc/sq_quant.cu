@@ -261,6 +261,30 @@ quant_rows_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
       }
     }
   }
+  if constexpr (OUTLIERS) {
+    if (ov.w_src != nullptr) {
+      // the weight's outlier columns, one thread per weight row: w_gathered[r, c] = w[r, idx[c]]
+      // for c < count, 0 up to the next multiple of 64, eight columns (16 bytes) per store
+      const int32_t cnt = __ldg(ov.count);
+      const int32_t padded = (cnt + 63) & ~63;
+      for (int64_t r = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; r < ov.w_rows;
+           r += static_cast<int64_t>(gridDim.x) * kThreads) {
+        const uint16_t* srow = ov.w_src + r * ov.w_ld;
+        uint4* drow = reinterpret_cast<uint4*>(ov.w_gathered + r * ov.ld_gathered);
+        for (int32_t c0 = 0; c0 < padded; c0 += 8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int32_t c = c0 + 2 * i;
+            const uint32_t lo = c < cnt ? srow[__ldg(ov.idx + c)] : 0u;
+            const uint32_t hi = c + 1 < cnt ? srow[__ldg(ov.idx + c + 1)] : 0u;
+            w[i] = lo | (hi << 16);
+          }
+          drow[c0 / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+  }
 }
 
 int num_sms() {

@@ -23,12 +23,55 @@ __device__ __forceinline__ int q8(float x, float r) {
   return __float_as_int(__fadd_rn(t, 12582912.0f));
 }
 
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic: two IEEE round-to-nearest operations per
+// instruction, each lane exactly the scalar result). Use them only where no packed multiply
+// feeds a packed add: such a pair was observed to execute as one fused multiply-add.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// q8 of two values at once (the products and the rounding add packed; the clamp between them
+// keeps the two from fusing).
+__device__ __forceinline__ void q8x2(float x0, float x1, uint64_t r2, int& q0, int& q1) {
+  float t0, t1;
+  f2_unpack(f2_mul(f2_pack(x0, x1), r2), t0, t1);
+  t0 = fminf(fmaxf(t0, -128.0f), 127.0f);
+  t1 = fminf(fmaxf(t1, -128.0f), 127.0f);
+  f2_unpack(f2_add(f2_pack(t0, t1), f2_pack(12582912.0f, 12582912.0f)), t0, t1);
+  q0 = __float_as_int(t0);
+  q1 = __float_as_int(t1);
+}
+
 __device__ __forceinline__ void store_q16(int8_t* dst, const float (&v)[16], float r) {
+  const uint64_t r2 = f2_pack(r, r);
+  int q[16];
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) q8x2(v[i], v[i + 1], r2, q[i], q[i + 1]);
   uint4 o;
-  o.x = pack4(q8(v[0], r), q8(v[1], r), q8(v[2], r), q8(v[3], r));
-  o.y = pack4(q8(v[4], r), q8(v[5], r), q8(v[6], r), q8(v[7], r));
-  o.z = pack4(q8(v[8], r), q8(v[9], r), q8(v[10], r), q8(v[11], r));
-  o.w = pack4(q8(v[12], r), q8(v[13], r), q8(v[14], r), q8(v[15], r));
+  o.x = pack4(q[0], q[1], q[2], q[3]);
+  o.y = pack4(q[4], q[5], q[6], q[7]);
+  o.z = pack4(q[8], q[9], q[10], q[11]);
+  o.w = pack4(q[12], q[13], q[14], q[15]);
   *reinterpret_cast<uint4*>(dst) = o;
 }
 

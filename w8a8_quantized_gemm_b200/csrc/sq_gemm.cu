@@ -55,6 +55,9 @@ struct Cfg {
   static constexpr int kStages = (192 * 1024) / kStageBytes;
   static constexpr int kAccCols = OUTLIERS ? 2 * BN : BN;  // per buffer: int32 acc (+ fp32 acc)
   static constexpr int kTmemCols = ACC_BUFS * kAccCols;
+  // with outlier operands but no outlier column at run time the int32 accumulator alone is
+  // needed, and the fp32 columns hold a second int32 buffer
+  static constexpr int kMaxBufs = (OUTLIERS && ACC_BUFS == 1) ? 2 : ACC_BUFS;
   static constexpr int kBarOffset = kStages * kStageBytes + kEpiSmem;
   static constexpr int kSmemBytes = kBarOffset + 256 /*barriers*/ + 1024 /*alignment slack*/;
   static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
@@ -320,8 +323,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint64_t* full = bars;
   uint64_t* empty = bars + C::kStages;
   uint64_t* tmem_full = bars + 2 * C::kStages;
-  uint64_t* tmem_empty = tmem_full + ACC_BUFS;
-  uint64_t* teardown = tmem_empty + ACC_BUFS;
+  uint64_t* tmem_empty = tmem_full + C::kMaxBufs;
+  uint64_t* teardown = tmem_empty + C::kMaxBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const Abort ab{abort_flag};
@@ -334,7 +337,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
-    for (int b = 0; b < ACC_BUFS; ++b) {
+    for (int b = 0; b < C::kMaxBufs; ++b) {
       mbar_init(tmem_full + b, 1);
       mbar_init(tmem_empty + b, kEpiWarps);
     }
@@ -365,6 +368,9 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const int num_units = p.num_units;
   int kb_o = 0;
   if constexpr (OUTLIERS) kb_o = (__ldg(p.o_count) + 63) / 64;
+  // accumulator buffers: double-buffered int32 when no outlier product is needed
+  const int acc_bufs = kb_o == 0 ? C::kMaxBufs : ACC_BUFS;
+  const uint32_t acc_cols = kb_o == 0 ? static_cast<uint32_t>(BN) : static_cast<uint32_t>(C::kAccCols);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -425,14 +431,14 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       uint32_t phase = 0;
       int it = 0;
       for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x, ++it) {
-        const int buf = it % ACC_BUFS;
-        const uint32_t acc_phase = (it / ACC_BUFS) & 1;
+        const int buf = it % acc_bufs;
+        const uint32_t acc_phase = (it / acc_bufs) & 1;
         if (!wait_or_abort(tmem_empty + buf, acc_phase ^ 1, p.wait_limit_ns, abort_flag)) {
           if (!*abort_flag) ab.raise(p.status, kErrMmaWait);
           break;
         }
         tc_fence_after();
-        const uint32_t d_i32 = tmem_base + buf * C::kAccCols;
+        const uint32_t d_i32 = tmem_base + buf * acc_cols;
         const uint32_t d_f32 = d_i32 + BN;
         const Unit w = unit_of(p, u);
         const int kb0 = w.kb0, kb_i8 = w.kb1;
@@ -488,8 +494,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     int ebuf = 0;
     int it = 0;
     for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++it) {
-      const int buf = it % ACC_BUFS;
-      const uint32_t acc_phase = (it / ACC_BUFS) & 1;
+      const int buf = it % acc_bufs;
+      const uint32_t acc_phase = (it / acc_bufs) & 1;
       // everything that does not need the accumulator is fetched before waiting for it
       const Unit w = unit_of(p, u);
       const int tile_mn = w.tile_mn;
@@ -526,7 +532,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       if (!ok) break;
       tc_fence_after();
       const uint32_t t_row =
-          tmem_base + buf * C::kAccCols + (static_cast<uint32_t>(quad * 32) << 16) + half * (BN / 2);
+          tmem_base + buf * acc_cols + (static_cast<uint32_t>(quad * 32) << 16) + half * (BN / 2);
       if (!w.is_split) {
         uint32_t packed[kChunks][16];
 #pragma unroll

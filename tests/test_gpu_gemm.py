@@ -95,7 +95,7 @@ def test_smoothquant_path_ragged(M, N, K, gran):
 
 def test_split_k_workspace_reused_across_calls():
     """The split-K arrival counters return to zero, so one workspace serves call after call."""
-    M, N, K = 16, 1024, 4096
+    M, N, K = 32, 1024, 4096  # swapped operands, 8 tiles each split 16 ways
     assert sq.sq_workspace_size(sq.SQ_OP_INT8_GEMM_DEQUANT, M, N, K) > 0
     rng = np.random.default_rng(11)
     ws = sq.workspace(sq.SQ_OP_INT8_GEMM_DEQUANT, M, N, K)

@@ -63,7 +63,8 @@ typedef enum {
   SQ_ERR_CUDA = -3,        /* a CUDA runtime / driver call failed (message has the code) */
   SQ_ERR_TIMEOUT = -4,     /* a bounded device-side wait gave up (see sq_sync_status) */
   SQ_ERR_WORKSPACE = -5,   /* ws NULL or smaller than sq_workspace_size() */
-  SQ_ERR_UNSUPPORTED = -6  /* no sm_100a device, or the library was built without it */
+  SQ_ERR_UNSUPPORTED = -6, /* no sm_100a device, or the library was built without it */
+  SQ_ERR_BOUNDS = -7       /* a device-side bounds guard fired (libsq_debug.so only; see sq_sync_status) */
 } sq_status;
 
 typedef enum { SQ_PER_TENSOR = 0, SQ_PER_CHANNEL = 1 } sq_gran;
@@ -337,7 +338,9 @@ SQ_API const char* sq_last_error(void);
 
 /* Synchronises `stream`, then reads and clears the current device's error word, which
  * kernels set when a bounded wait gives up (a device-side stall or lost arrival) instead
- * of spinning forever. Returns SQ_OK, SQ_ERR_TIMEOUT or SQ_ERR_CUDA. */
+ * of spinning forever, and, in the debug build libsq_debug.so (same ABI, kernels compiled
+ * with device-side bounds guards that skip and record an out-of-range access), when a guard
+ * fires. Returns SQ_OK, SQ_ERR_TIMEOUT, SQ_ERR_BOUNDS or SQ_ERR_CUDA. */
 SQ_API sq_status sq_sync_status(sq_stream_t stream);
 
 /* Library version string and the compute capability it was built for ("sm_100a"). */

@@ -139,3 +139,13 @@ def test_variant_validation():
     lneed = sq.sq_workspace_size(sq.SQ_OP_LLMINT8, 16, 16, 64)
     assert L.llmint8_decomposed_linear_ex(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 16, 16, 64, None, None, None,
                                           FAKE, lneed, None) == sq.SQ_ERR_INVALID
+
+
+def test_debug_build_exports_the_same_symbols():
+    """libsq_debug.so (bounds guards) carries the ABI of libsq.so (plus the device-link
+    registration stubs that relocatable device code adds)."""
+    from w8a8_quantized_gemm_b200 import build as _b
+    out = os.popen(f"nm -D --defined-only {_b.LIB_DEBUG}").read().split("\n")
+    exported = {l.split()[-1] for l in out if " T " in l}
+    assert exported >= set(_declared())
+    assert all(n in _declared() or n.startswith("__cuda") for n in exported)

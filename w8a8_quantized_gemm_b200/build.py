@@ -1,8 +1,9 @@
-"""Build libsq.so (the CUDA kernels + C ABI) in-tree for sm_100a with nvcc.
+"""Build libsq.so (the CUDA kernels + C ABI) in-tree for sm_100a with nvcc, and its
+bounds-guard twin libsq_debug.so (same ABI; kernels record and skip out-of-range accesses).
 
-Usage: ``python -m w8a8_quantized_gemm_b200.build [--force] [--verbose]``.
-Object files go to ``_build/`` at the repository root; the shared library is
-written next to this file so that the Python binding finds it.
+Usage: ``python -m w8a8_quantized_gemm_b200.build [--force] [--verbose] [--no-debug]``.
+Object files go to ``_build/`` (``_build/debug/``) at the repository root; the shared
+libraries are written next to this file so that the Python binding finds them.
 """
 from __future__ import annotations
 
@@ -19,6 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsq.so")
+LIB_DEBUG = os.path.join(PKG, "libsq_debug.so")
 
 SOURCES = ["sq_api.cu", "sq_reduce.cu", "sq_quant.cu", "sq_outlier.cu", "sq_gemm.cu", "sq_noalloc.cu",
            "sq_variants.cu", "sq_gemv.cu"]
@@ -47,16 +49,17 @@ def _stale(target: str, deps: list) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def _build_flavor(lib: str, obj_dir: str, extra: list, link_extra: list, force: bool, verbose: bool,
+                  ptxas_info: bool) -> str:
+    os.makedirs(obj_dir, exist_ok=True)
     cc = nvcc()
     objs, jobs = [], []
     for s in SOURCES:
         src = os.path.join(CSRC, s)
-        obj = os.path.join(BUILD, s.replace(".cu", ".o"))
+        obj = os.path.join(obj_dir, s.replace(".cu", ".o"))
         objs.append(obj)
         if force or ptxas_info or _stale(obj, _deps(src)):
-            cmd = [cc, *ARCH, *NVCC_FLAGS, *(["-Xptxas", "-v"] if ptxas_info else []), "-c", src, "-o", obj]
+            cmd = [cc, *ARCH, *NVCC_FLAGS, *extra, *(["-Xptxas", "-v"] if ptxas_info else []), "-c", src, "-o", obj]
             jobs.append(cmd)
     if jobs:
         with cf.ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 4)) as ex:
@@ -67,13 +70,24 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
                     sys.stderr.write(" ".join(j) + "\n" + r.stdout + r.stderr)
                 if r.returncode:
                     raise RuntimeError(f"nvcc failed for {j[-3]}")
-    if force or jobs or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
-        cmd = [cc, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-ldl", "-lrt", "-lpthread"]
+    if force or jobs or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
+        cmd = [cc, *ARCH, "-shared", *link_extra, "-o", tmp, *objs, "-lcudart_static", "-ldl", "-lrt", "-lpthread"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode:
             raise RuntimeError("link failed:\n" + r.stdout + r.stderr)
-        os.replace(tmp, LIB)
+        os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, debug: bool = True) -> str:
+    """Build libsq.so and (with `debug`) libsq_debug.so: the same sources with device-side
+    bounds guards (SQ_DEBUG_GUARDS; relocatable device code so that every unit reaches the
+    one error word). Returns the product library's path."""
+    _build_flavor(LIB, BUILD, [], [], force, verbose, ptxas_info)
+    if debug:
+        _build_flavor(LIB_DEBUG, os.path.join(BUILD, "debug"), ["-DSQ_DEBUG_GUARDS", "-rdc=true"], ["-rdc=true"],
+                      force, verbose, False)
     return LIB
 
 
@@ -82,5 +96,6 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true", help="print registers / spills / smem per kernel")
+    ap.add_argument("--no-debug", action="store_true", help="skip the bounds-guard build libsq_debug.so")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose, ptxas_info=a.ptxas_info))
+    print(build(force=a.force, verbose=a.verbose, ptxas_info=a.ptxas_info, debug=not a.no_debug))

@@ -525,6 +525,8 @@ sq_status sq_sync_status(sq_stream_t stream) {
     const unsigned int zero = 0;
     e = cudaMemcpyToSymbol(sq::g_status_word, &zero, sizeof zero);
     if (e != cudaSuccess) return cuda_fail(e, "sq_sync_status: clear status word");
+    if (word & sq::kErrBounds)
+      return fail(SQ_ERR_BOUNDS, "device bounds guard fired (status bits 0x%x)", word);
     return fail(SQ_ERR_TIMEOUT, "device wait timed out (status bits 0x%x: 1 producer, 2 mma, 4 epilogue, 8 teardown)",
                 word);
   }

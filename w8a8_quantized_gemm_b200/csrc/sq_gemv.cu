@@ -81,7 +81,7 @@ gemv_i8_kernel(const int8_t* __restrict__ Xq, const int8_t* __restrict__ Wq, con
       for (int o = 16; o > 0; o >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], o);
     }
     // lane m finishes token m of channel n
-    if (lane < M) {
+    if (lane < M && SQ_GUARD(n < N)) {
       int a = acc[0];
 #pragma unroll
       for (int m = 1; m < MT; ++m)

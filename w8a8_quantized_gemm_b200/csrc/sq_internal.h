@@ -14,6 +14,7 @@ enum : unsigned int {
   kErrMmaWait = 2u,
   kErrEpilogueWait = 4u,
   kErrTeardownWait = 8u,
+  kErrBounds = 16u,  // a device-side bounds guard fired (builds with SQ_DEBUG_GUARDS only)
 };
 
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s per wait
@@ -55,6 +56,21 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
 }
 
 #ifdef __CUDACC__
+// Device-side bounds guards. In the SQ_DEBUG_GUARDS build (libsq_debug.so) SQ_GUARD(c) checks
+// c, and when it is false records kErrBounds in the device error word (sq_sync_status then
+// reports SQ_ERR_BOUNDS) so that the caller skips the access; in the product build it is the
+// constant true and costs nothing.
+#ifdef SQ_DEBUG_GUARDS
+extern __device__ unsigned int g_status_word;
+__device__ __forceinline__ bool guard_ok(bool c) {
+  if (!c) atomicOr(&g_status_word, kErrBounds);
+  return c;
+}
+#define SQ_GUARD(c) (::sq::guard_ok(c))
+#else
+#define SQ_GUARD(c) true
+#endif
+
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

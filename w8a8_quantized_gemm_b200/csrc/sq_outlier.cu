@@ -102,7 +102,8 @@ outlier_mask_kernel(const float* __restrict__ amax, int64_t K, float threshold_v
       int32_t pos = excl;
       while (rest) {
         const int i = __ffs(rest) - 1;
-        idx[pos++] = static_cast<int32_t>(word * 32 + i);
+        if (SQ_GUARD(pos < K && word * 32 + i < K)) idx[pos] = static_cast<int32_t>(word * 32 + i);
+        ++pos;
         rest &= rest - 1u;
       }
     }

@@ -50,7 +50,7 @@ __device__ __forceinline__ void finish_chunk(const uint4 (&r)[2], int64_t row, i
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         if ((sk >> i) & 1u) {
-          if (gather) ov.gathered[row * ov.ld_gathered + pos] = h[i];
+          if (gather && SQ_GUARD(pos >= 0 && pos < ov.ld_gathered)) ov.gathered[row * ov.ld_gathered + pos] = h[i];
           ++pos;
           v[i] = 0.0f;
         }
@@ -256,7 +256,8 @@ quant_rows_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
           // zero the padding of the gathered row up to the next multiple of 64 columns
           const int32_t cnt = __ldg(ov.count);
           const int32_t padded = (cnt + 63) & ~63;
-          for (int32_t c = cnt + t; c < padded; c += TPR) ov.gathered[row * ov.ld_gathered + c] = 0;
+          for (int32_t c = cnt + t; c < padded; c += TPR)
+            if (SQ_GUARD(c < ov.ld_gathered)) ov.gathered[row * ov.ld_gathered + c] = 0;
         }
       }
     }
@@ -276,11 +277,13 @@ quant_rows_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int32_t c = c0 + 2 * i;
-            const uint32_t lo = c < cnt ? srow[__ldg(ov.idx + c)] : 0u;
-            const uint32_t hi = c + 1 < cnt ? srow[__ldg(ov.idx + c + 1)] : 0u;
+            const int32_t jl = c < cnt ? __ldg(ov.idx + c) : 0;
+            const int32_t jh = c + 1 < cnt ? __ldg(ov.idx + c + 1) : 0;
+            const uint32_t lo = (c < cnt && SQ_GUARD(jl >= 0 && jl < ov.w_ld)) ? srow[jl] : 0u;
+            const uint32_t hi = (c + 1 < cnt && SQ_GUARD(jh >= 0 && jh < ov.w_ld)) ? srow[jh] : 0u;
             w[i] = lo | (hi << 16);
           }
-          drow[c0 / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+          if (SQ_GUARD(c0 + 8 <= ov.ld_gathered)) drow[c0 / 8] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
     }

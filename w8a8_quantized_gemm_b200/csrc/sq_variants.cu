@@ -225,7 +225,7 @@ norm_quant_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
 #pragma unroll
       for (int c = 0; c < CHUNKS; ++c) {
         const int64_t k = c * step + t * 16;
-        if (k < K) store_q16(qrow + k, x[c], r);
+        if (k < K && SQ_GUARD(k + 16 <= K)) store_q16(qrow + k, x[c], r);
       }
     }
   }
@@ -373,7 +373,7 @@ select_rank_kernel(const unsigned long long* __restrict__ hist, unsigned long lo
     unsigned long long run = before;
     for (int i = 0; i < kPer; ++i) {
       run += hist[t * kPer + i];
-      if (run >= rank) {
+      if (run >= rank && SQ_GUARD(t * kPer + i < kBins)) {
         *out = __uint_as_float(static_cast<uint32_t>(t * kPer + i) << 16);
         break;
       }

@@ -14,10 +14,12 @@ import os
 from typing import Optional
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsq.so")
+# SQ_LIB_PATH selects another build of the same ABI (the bounds-guard build libsq_debug.so)
+LIB_PATH = os.environ.get("SQ_LIB_PATH") or os.path.join(_HERE, "libsq.so")
 
 SQ_OK, SQ_ERR_INVALID, SQ_ERR_ALIGN, SQ_ERR_CUDA, SQ_ERR_TIMEOUT, SQ_ERR_WORKSPACE, SQ_ERR_UNSUPPORTED = \
     0, -1, -2, -3, -4, -5, -6
+SQ_ERR_BOUNDS = -7
 SQ_PER_TENSOR, SQ_PER_CHANNEL = 0, 1
 SQ_OP_SMOOTH_QUANT_WEIGHT, SQ_OP_INT8_GEMM_DEQUANT, SQ_OP_LLMINT8 = 1, 2, 3
 SQ_OP_QUANT_ACT_PER_TENSOR, SQ_OP_MEAN_STD_THRESHOLD, SQ_OP_ABS_PERCENTILE = 4, 5, 6

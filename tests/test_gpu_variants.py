@@ -287,3 +287,59 @@ def test_mean_std_threshold(M, K, k):
     assert abs(gm - omean) <= 1e-11 * max(1.0, abs(omean), osd)
     assert abs(gs - osd) <= 1e-11 * max(osd, 1e-300) or osd == 0.0
     assert _ulps(host(thr), othr).max() <= 1
+
+
+# --------------------------------------------------------------------------- strided inputs
+def test_strided_inputs_every_row_kernel():
+    """Column slices of a wider matrix (leading dimension 1024 > K = 528): the row kernels
+    read through ld, and every result equals the oracle's on the contiguous slice."""
+    rng = np.random.default_rng(31)
+    M, LD, K, off = 37, 1024, 528, 64
+    full = wl.f32_to_bf16_bits(rng.normal(0.2, 1.5, (M, LD)).astype(np.float32))
+    wfull = wl.f32_to_bf16_bits(rng.normal(0, 0.02, (96, LD)).astype(np.float32))
+    X = dev_bf16(full)[:, off:off + K]
+    W = dev_bf16(wfull)[:, off:off + K]
+    Xc = np.ascontiguousarray(full[:, off:off + K])
+    Wc = np.ascontiguousarray(wfull[:, off:off + K])
+    inv_s = rng.uniform(0.3, 2.0, K).astype(np.float32)
+    inv_t = torch.from_numpy(inv_s).cuda()
+    # per-token quantization
+    Xq, d = empty((M, K), torch.int8), empty(M, torch.float32)
+    sq.sq_quant_act_per_token(X, inv_t, Xq, d)
+    sq.sq_sync_status()
+    oq, od = oracle.quant_act_per_token(Xc, inv_s)
+    assert np.array_equal(host(Xq), oq) and np.array_equal(host(d), od)
+    # smoothing factors and both weight granularities
+    amax = torch.from_numpy(oracle.act_channel_absmax(Xc)).cuda()
+    s, i = empty(K, torch.float32), empty(K, torch.float32)
+    sq.sq_smooth_scale(amax, W, 0.5, s, i)
+    sq.sq_sync_status()
+    os_, _ = oracle.smooth_scale(host(amax), Wc, 0.5)
+    assert _ulps(host(s), os_).max() <= 1
+    for gran in (sq.SQ_PER_CHANNEL, sq.SQ_PER_TENSOR):
+        Wq, e = empty((96, K), torch.int8), empty(96 if gran == sq.SQ_PER_CHANNEL else 1, torch.float32)
+        sq.sq_smooth_quant_weight(W, s, gran, Wq, e, sq.workspace(sq.SQ_OP_SMOOTH_QUANT_WEIGHT, 0, 96, K))
+        sq.sq_sync_status()
+        owq, oe = oracle.smooth_quant_weight(Wc, host(s), gran)
+        assert np.array_equal(host(Wq), owq) and np.array_equal(host(e), oe)
+    # fused LayerNorm, asymmetric, per-tensor, mean/std
+    g = wl.f32_to_bf16_bits(rng.uniform(0.5, 1.5, K).astype(np.float32))
+    st = empty((M, 2), torch.float32)
+    sq.sq_norm_smooth_quant(X, sq.SQ_NORM_LAYER, dev_bf16(g), None, 1e-5, inv_t, Xq, d, st)
+    sq.sq_sync_status()
+    cq, cd, _ = oracle.norm_smooth_quant(Xc, oracle.NORM_LAYER, g, None, 1e-5, inv_s, stats=host(st))
+    assert np.array_equal(host(Xq), cq) and np.array_equal(host(d), cd)
+    z = empty(M, torch.int32)
+    sq.sq_quant_act_per_token_asym(X, inv_t, Xq, d, z)
+    sq.sq_sync_status()
+    aq, ad, az = oracle.quant_act_per_token_asym(Xc, inv_s)
+    assert np.array_equal(host(Xq), aq) and np.array_equal(host(d), ad) and np.array_equal(host(z), az)
+    d1 = empty(1, torch.float32)
+    sq.sq_quant_act_per_tensor(X, inv_t, Xq, d1, None, sq.workspace(sq.SQ_OP_QUANT_ACT_PER_TENSOR, M, 0, K))
+    sq.sq_sync_status()
+    pq, pd = oracle.quant_act_per_tensor(Xc, inv_s)
+    assert np.array_equal(host(Xq), pq) and np.array_equal(host(d1), pd)
+    thr = empty(1, torch.float32)
+    sq.sq_act_mean_std_threshold(X, 3.0, thr, None, sq.workspace(sq.SQ_OP_MEAN_STD_THRESHOLD, M, 0, K))
+    sq.sq_sync_status()
+    assert _ulps(host(thr), oracle.mean_std_threshold(Xc, 3.0)[0]).max() <= 1

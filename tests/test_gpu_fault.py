@@ -13,8 +13,9 @@ from _gpu import empty, host
 pytestmark = pytest.mark.gpu
 
 
-def test_withheld_stage_times_out_and_context_survives():
-    M, N, K = 256, 512, 1024
+# one CTA per tile, and CTA pairs on 256 x 256 tiles (the abort reaches the other CTA too)
+@pytest.mark.parametrize("M,N,K", [(256, 512, 1024), (2433, 1800, 272)])
+def test_withheld_stage_times_out_and_context_survives(M, N, K):
     rng = np.random.default_rng(0)
     xq = rng.integers(-127, 128, size=(M, K), dtype=np.int8)
     wq = rng.integers(-127, 128, size=(N, K), dtype=np.int8)

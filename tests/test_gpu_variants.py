@@ -102,7 +102,7 @@ def test_smooth_scale_normalised():
 
 # --------------------------------------------------------------------------- GEMM variants
 GEMM_EX_SHAPES = [(1, 8, 16), (5, 24, 48), (64, 4096, 4096), (130, 72, 144), (300, 9480, 528), (257, 1000, 528),
-                  (1024, 2048, 1024), (37, 9736, 256)]
+                  (1024, 2048, 1024), (37, 9736, 256), (2433, 1800, 272)]
 
 
 def _codes(rng, M, N, K):

@@ -47,10 +47,12 @@ constexpr int kStageTileBytes = 32 * 32 * 2;  // one 32-row x 32-column bf16 out
 constexpr int kEpiBufs = 2;                   // per epilogue warp
 constexpr int kEpiSmem = kEpiWarps * kEpiBufs * kStageTileBytes;
 
-template <int BN, bool OUTLIERS, int ACC_BUFS>
+// PAIR: a CTA pair computes one 256 x BN tile; each CTA stages its 128 rows of A and half
+// of the BN rows of B, so a stage holds 32 KB instead of 48 and the ring gets 6 stages.
+template <int BN, bool OUTLIERS, int ACC_BUFS, bool PAIR = false>
 struct Cfg {
   static constexpr int kStageA = kBM * kBK;
-  static constexpr int kStageB = BN * kBK;
+  static constexpr int kStageB = (PAIR ? BN / 2 : BN) * kBK;
   static constexpr int kStageBytes = kStageA + kStageB;
   static constexpr int kStages = (192 * 1024) / kStageBytes;
   static constexpr int kAccCols = OUTLIERS ? 2 * BN : BN;  // per buffer: int32 acc (+ fp32 acc)
@@ -97,9 +99,11 @@ struct Params {
 
 struct Abort {
   volatile int* flag;
+  uint32_t peer_flag;  // the other CTA's flag (shared::cluster address) in a CTA pair, else 0
   __device__ void raise(unsigned int* status, unsigned int bit) const {
     atomicOr(status, bit);
     *flag = 1;
+    if (peer_flag != 0) st_cluster_u32(peer_flag, 1u);
   }
 };
 
@@ -309,12 +313,15 @@ __device__ __forceinline__ void store_box(const uint32_t (&v)[16], uint8_t* stag
   ebuf ^= 1;
 }
 
-template <int BN, bool OUTLIERS, int ACC_BUFS, bool SWAP, bool ASYM>
+template <int BN, bool OUTLIERS, int ACC_BUFS, bool SWAP, bool ASYM, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmXo, const __grid_constant__ CUtensorMap tmWo,
                  const __grid_constant__ CUtensorMap tmY, const Params p) {
-  using C = Cfg<BN, OUTLIERS, ACC_BUFS>;
+  using C = Cfg<BN, OUTLIERS, ACC_BUFS, PAIR>;
+  static_assert(!PAIR || (!SWAP && !OUTLIERS && BN == 256), "CTA pairs: plain 256 x 256 tiles");
+  // rows of A per output tile: one CTA's 128, or a pair's 256 (this CTA's half at rank * 128)
+  constexpr int kTileM = PAIR ? 2 * kBM : kBM;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
@@ -327,10 +334,15 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint64_t* teardown = tmem_empty + C::kMaxBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const Abort ab{abort_flag};
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;  // the pair's MMA issuer (always true for a single CTA)
+  const Abort ab{abort_flag, PAIR ? mapa_shared(const_cast<int*>(abort_flag), rank ^ 1u) : 0u};
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // work units of this CTA (a pair walks them together)
+  const int u_first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int u_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -339,7 +351,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
     for (int b = 0; b < C::kMaxBufs; ++b) {
       mbar_init(tmem_full + b, 1);
-      mbar_init(tmem_empty + b, kEpiWarps);
+      mbar_init(tmem_empty + b, PAIR ? 2 * kEpiWarps : kEpiWarps);
     }
     mbar_init(teardown, 1);
     *abort_flag = 0;
@@ -354,11 +366,19 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync();  // both CTAs' barriers initialised before any remote arrive or copy
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // set-up done: from here on global memory written by the previous kernel is read
@@ -380,10 +400,10 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       uint32_t issued_mask = 0;      // stages that received at least one load
       uint32_t issued_parity = 0;    // parity of the last load issued into each stage
       bool withheld = false;
-      for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
+      for (int u = u_first; u < num_units && !*abort_flag; u += u_step) {
         const Unit w = unit_of(p, u);
-        const int m0 = (w.tile_mn % p.num_m_tiles) * kBM;
-        const int n0 = (w.tile_mn / p.num_m_tiles) * BN;
+        const int m0 = (w.tile_mn % p.num_m_tiles) * kTileM + static_cast<int>(rank) * kBM;
+        const int n0 = (w.tile_mn / p.num_m_tiles) * BN + (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
         const int kb0 = w.kb0, kb_i8 = w.kb1;
         const int kb_total = kb_i8 + kb_o;
         for (int kb = kb0; kb < kb_total; ++kb) {
@@ -396,14 +416,22 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           } else {
             uint8_t* sa = stage_base + stage * C::kStageBytes;
             uint8_t* sb = sa + C::kStageA;
-            mbar_arrive_expect_tx(full + stage, C::kStageBytes);
-            if (kb < kb_i8) {
-              tma_load_2d(sa, &tmA, full + stage, kb * kBK, m0, kEvictNormal);
-              tma_load_2d(sb, &tmB, full + stage, kb * kBK, n0, kEvictNormal);
+            if constexpr (PAIR) {
+              // both CTAs' halves complete on the even CTA's barrier, which expects them all
+              if (leader) mbar_arrive_expect_tx(full + stage, 2 * C::kStageBytes);
+              const uint32_t fb = mapa_shared(full + stage, 0);
+              tma_load_2d_pair(sa, &tmA, fb, kb * kBK, m0, kEvictNormal);
+              tma_load_2d_pair(sb, &tmB, fb, kb * kBK, n0, kEvictNormal);
             } else {
-              const int ko = (kb - kb_i8) * (kBK / 2);
-              tma_load_2d(sa, &tmXo, full + stage, ko, m0, kEvictNormal);
-              tma_load_2d(sb, &tmWo, full + stage, ko, n0, kEvictNormal);
+              mbar_arrive_expect_tx(full + stage, C::kStageBytes);
+              if (kb < kb_i8) {
+                tma_load_2d(sa, &tmA, full + stage, kb * kBK, m0, kEvictNormal);
+                tma_load_2d(sb, &tmB, full + stage, kb * kBK, n0, kEvictNormal);
+              } else {
+                const int ko = (kb - kb_i8) * (kBK / 2);
+                tma_load_2d(sa, &tmXo, full + stage, ko, m0, kEvictNormal);
+                tma_load_2d(sb, &tmWo, full + stage, ko, n0, kEvictNormal);
+              }
             }
             issued_mask |= 1u << stage;
             issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -414,9 +442,11 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           }
         }
       }
-      // drain: every load this thread issued must have landed before the CTA exits
+      // drain: every load this thread issued must have landed before the CTA exits (a
+      // pair's odd CTA counts its copies on the even CTA's barriers, which the even CTA
+      // drains before the final cluster barrier)
       for (int s = 0; s < C::kStages; ++s) {
-        if ((issued_mask >> s) & 1u) {
+        if (leader && ((issued_mask >> s) & 1u)) {
           if (!mbar_wait_bounded(full + s, (issued_parity >> s) & 1u, p.wait_limit_ns))
             ab.raise(p.status, kErrTeardownWait);
         }
@@ -424,13 +454,17 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdescI8 = idesc_i8_s32(kBM, BN);
+    if (lane == 0 && leader) {
+      constexpr uint32_t kIdescI8 = idesc_i8_s32(kTileM, BN);
       constexpr uint32_t kIdescBf16 = idesc_bf16_f32(kBM, BN);
+      // a pair's commits go to the barrier in each CTA (shared::cluster addresses)
+      const uint32_t empty_c0 = PAIR ? mapa_shared(empty, 0) : 0u, empty_c1 = PAIR ? mapa_shared(empty, 1) : 0u;
+      const uint32_t tfull_c0 = PAIR ? mapa_shared(tmem_full, 0) : 0u;
+      const uint32_t tfull_c1 = PAIR ? mapa_shared(tmem_full, 1) : 0u;
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
-      for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x, ++it) {
+      for (int u = u_first; u < num_units && !*abort_flag; u += u_step, ++it) {
         const int buf = it % acc_bufs;
         const uint32_t acc_phase = (it / acc_bufs) & 1;
         if (!wait_or_abort(tmem_empty + buf, acc_phase ^ 1, p.wait_limit_ns, abort_flag)) {
@@ -453,7 +487,14 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           tc_fence_after();
           const uint32_t a_addr = smem_u32(stage_base + stage * C::kStageBytes);
           const uint32_t b_addr = a_addr + C::kStageA;
-          if (kb < kb_i8) {
+          if constexpr (PAIR) {
+#pragma unroll
+            for (int k = 0; k < kBK / 32; ++k)
+              mma_i8_pair(d_i32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescI8,
+                          (kb != kb0 || k != 0) ? 1u : 0u);
+            mma_commit_pair(empty_c0 + 8u * stage);
+            mma_commit_pair(empty_c1 + 8u * stage);
+          } else if (kb < kb_i8) {
 #pragma unroll
             for (int k = 0; k < kBK / 32; ++k)
               mma_i8(d_i32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescI8,
@@ -465,17 +506,26 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
               mma_f16(d_f32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescBf16,
                       (ko | k) != 0);
           }
-          mma_commit(empty + stage);
+          if constexpr (!PAIR) mma_commit(empty + stage);
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        mma_commit(tmem_full + buf);
+        if constexpr (PAIR) {
+          mma_commit_pair(tfull_c0 + 8u * buf);
+          mma_commit_pair(tfull_c1 + 8u * buf);
+        } else {
+          mma_commit(tmem_full + buf);
+        }
       }
-      // all MMAs issued by this thread complete before TMEM is released
-      mma_commit(teardown);
+      // all MMAs issued by this thread complete before TMEM is released (in both CTAs of a
+      // pair: the odd CTA frees its TMEM only after the final cluster barrier)
+      if constexpr (PAIR)
+        mma_commit_pair(smem_u32(teardown));
+      else
+        mma_commit(teardown);
       if (!mbar_wait_bounded(teardown, 0, p.wait_limit_ns)) ab.raise(p.status, kErrTeardownWait);
     }
   } else {
@@ -493,14 +543,16 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     uint8_t* stage_tiles = epi_base + (warp - 2) * kEpiBufs * kStageTileBytes;
     int ebuf = 0;
     int it = 0;
-    for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++it) {
+    // a pair's odd CTA hands the accumulator back on the even CTA's barrier
+    const uint32_t tempty_c0 = PAIR ? mapa_shared(tmem_empty, 0) : 0u;
+    for (int u = u_first; u < num_units; u += u_step, ++it) {
       const int buf = it % acc_bufs;
       const uint32_t acc_phase = (it / acc_bufs) & 1;
       // everything that does not need the accumulator is fetched before waiting for it
       const Unit w = unit_of(p, u);
       const int tile_mn = w.tile_mn;
       const int split = w.split;
-      const int64_t m_tile0 = static_cast<int64_t>(tile_mn % p.num_m_tiles) * kBM;
+      const int64_t m_tile0 = static_cast<int64_t>(tile_mn % p.num_m_tiles) * kTileM + rank * kBM;
       const int64_t r = m_tile0 + row;  // this thread's tile row (output row, or channel if swapped)
       const int64_t box_row0 = m_tile0 + quad * 32;
       const bool rows_live = box_row0 < p.rows;  // uniform across the warp
@@ -562,7 +614,12 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // the accumulator is no longer needed: hand it back before storing
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(tmem_empty + buf);
+        if (lane == 0) {
+          if constexpr (PAIR)
+            mbar_arrive_remote(tempty_c0 + 8u * buf);
+          else
+            mbar_arrive(tmem_empty + buf);
+        }
         if (rows_live) {
 #pragma unroll
           for (int c = 0; c < kChunks; ++c) {
@@ -645,9 +702,17 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
   __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync();  // no copy, MMA or remote arrive into either CTA is outstanding past here
+  else
+    __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+  if (warp == 1) {
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else
+      tmem_dealloc(tmem_base, C::kTmemCols);
+  }
 }
 
 // ---------------------------------------------------------------- host side
@@ -695,6 +760,7 @@ int num_sms() {
 
 struct Plan {
   bool swap;         // weight rows on the 128-row MMA operand, tokens on the BN columns
+  bool pair;         // CTA pairs on 256 x 256 tiles
   int bn;
   int num_full;      // whole-tile units
   int tail_tiles;    // tiles split along K
@@ -708,7 +774,9 @@ constexpr int64_t kSwapMaxM = 64;  // token counts that fit one 64-column tile
 
 // Operand roles: up to 64 tokens (and no outlier product) swap the operands, so the weight
 // rows fill the 128-row MMA operand and the tokens one 64-column tile. Otherwise the tile
-// width is the widest of 256/128/64 whose tile count covers the SMs. Problems with fewer
+// width is the widest of 256/128/64 whose tile count covers the SMs; 256-wide tiles become
+// 256 x 256 CTA-pair tiles when those still cover the SM pairs (each CTA then stages
+// two thirds of the bytes per k-block of a one-CTA 128 x 256 tile). Problems with fewer
 // tiles than half the SMs (small M, or a swapped decode shape) split every tile along K
 // into S parts whose exact int32 partials meet in the workspace. (Splitting only the tiles
 // of a last partial wave was measured slower on the 2048 x 11008 x 4096 shape, so whole
@@ -720,11 +788,18 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool outliers) {
   const int64_t m_t = (rows + kBM - 1) / kBM;
   const int64_t kb = (K + kBK - 1) / kBK;
   auto tiles = [&](int bn) { return m_t * ((cols + bn - 1) / bn); };
-  Plan pl{swap, 64, 0, 0, 1, static_cast<int>(kb)};
+  Plan pl{swap, false, 64, 0, 0, 1, static_cast<int>(kb)};
   if (swap) {
     pl.bn = 64;
   } else if (tiles(256) >= kPlanSms) {
     pl.bn = 256;
+    // CTA pairs when the 256 x 256 tiles still give every pair of SMs a tile
+    const int64_t pair_tiles = ((rows + 2 * kBM - 1) / (2 * kBM)) * ((cols + 255) / 256);
+    if (!outliers && pair_tiles >= kPlanSms / 2) {
+      pl.pair = true;
+      pl.num_full = static_cast<int>(pair_tiles);
+      return pl;
+    }
   } else if (tiles(128) >= kPlanSms) {
     pl.bn = 128;
   }
@@ -743,9 +818,10 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool outliers) {
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
-template <int BN, bool OUTLIERS, int ACC_BUFS, bool SWAP, bool ASYM = false>
+template <int BN, bool OUTLIERS, int ACC_BUFS, bool SWAP, bool ASYM = false, bool PAIR = false>
 cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const char** why) {
-  using C = Cfg<BN, OUTLIERS, ACC_BUFS>;
+  using C = Cfg<BN, OUTLIERS, ACC_BUFS, PAIR>;
+  auto kernel = w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS, SWAP, ASYM, PAIR>;
   CUtensorMap tmA{}, tmB{}, tmXo{}, tmWo{}, tmY{};
   const uint64_t K = static_cast<uint64_t>(a.K);
   // A: the 128-row operand (Xq, or Wq when swapped); B: the BN-row operand
@@ -754,7 +830,7 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   const int64_t rows = SWAP ? a.N : a.M;
   const int64_t cols = SWAP ? a.M : a.N;
   if (!make_operand_map(&tmA, a_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, rows, K, kBM) ||
-      !make_operand_map(&tmB, b_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, cols, K, BN)) {
+      !make_operand_map(&tmB, b_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, cols, K, PAIR ? BN / 2 : BN)) {
     *why = "cuTensorMapEncodeTiled failed for the int8 operands";
     return cudaErrorInvalidValue;
   }
@@ -779,8 +855,7 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   cudaGetDevice(&dev);
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_done.load() & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS, SWAP, ASYM>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) {
       *why = "cudaFuncSetAttribute(MaxDynamicSharedMemorySize) failed";
       return e;
@@ -800,7 +875,8 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   p.N = a.N;
   p.rows = rows;
   p.cols = cols;
-  p.num_m_tiles = static_cast<int>((rows + kBM - 1) / kBM);
+  constexpr int kTileM = PAIR ? 2 * kBM : kBM;
+  p.num_m_tiles = static_cast<int>((rows + kTileM - 1) / kTileM);
   p.num_n_tiles = static_cast<int>((cols + BN - 1) / BN);
   p.num_kb = static_cast<int>((a.K + kBK - 1) / kBK);
   p.num_full = pl.num_full;
@@ -818,12 +894,13 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   p.status = device_status_word();
   p.wait_limit_ns = a.wait_limit_ns;
   p.fault = a.fault;
-  const int grid = std::min(p.num_units, num_sms());
+  // one persistent CTA per SM (a pair per two SMs)
+  const int grid = PAIR ? 2 * std::min(p.num_units, num_sms() / 2) : std::min(p.num_units, num_sms());
   // short, latency-bound launches (swapped or K-split plans) overlap their set-up with
   // the previous kernel's tail
   const bool programmatic = SWAP || pl.tail_tiles > 0;
-  return launch_kernel(w8a8_gemm_kernel<BN, OUTLIERS, ACC_BUFS, SWAP, ASYM>, dim3(grid), dim3(kThreads), C::kSmemBytes,
-                       stream, programmatic, tmA, tmB, tmXo, tmWo, tmY, p);
+  return launch_kernel_clustered(kernel, dim3(grid), dim3(kThreads), C::kSmemBytes, stream, programmatic,
+                                 PAIR ? 2u : 1u, tmA, tmB, tmXo, tmWo, tmY, p);
 }
 
 }  // namespace
@@ -846,6 +923,10 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream, const char** why
     if (pl.bn == 256) return run<256, true, 1, false>(a, pl, stream, why);
     if (pl.bn == 128) return run<128, true, 2, false>(a, pl, stream, why);
     return run<64, true, 2, false>(a, pl, stream, why);
+  }
+  if (pl.pair) {
+    if (a.x_zero != nullptr) return run<256, false, 2, false, true, true>(a, pl, stream, why);
+    return run<256, false, 2, false, false, true>(a, pl, stream, why);
   }
   if (a.x_zero != nullptr) {
     if (pl.swap) return run<64, false, 2, true, true>(a, pl, stream, why);

@@ -38,21 +38,35 @@ int record_error(int st, const char* msg);
 // Only short, latency-bound launches take it: measured on the whole SmoothQuant +
 // LLM.int8 step (2048 x 11008 x 4096), setting it on every launch made the step 1-3%
 // slower, while a 4096 x 4096 decode GEMM gains ~0.8 us (of ~10.6).
+// `cluster_x` > 1 groups consecutive CTAs into clusters of that many (CTA pairs: 2).
 template <typename... KArgs, typename... Args>
-cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                          bool programmatic, Args&&... args) {
+cudaError_t launch_kernel_clustered(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                    bool programmatic, unsigned cluster_x, Args&&... args) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = programmatic ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (cluster_x > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
   note_launch();
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          bool programmatic, Args&&... args) {
+  return launch_kernel_clustered(kernel, grid, block, smem, stream, programmatic, 1u, std::forward<Args>(args)...);
 }
 
 #ifdef __CUDACC__

@@ -145,10 +145,10 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, ui
   }
 }
 
+// bf16_rne(lo) in the low half, bf16_rne(hi) in the high half (one conversion instruction).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-  const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-  return l | (h << 16);
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
 
 // Per-warp column constants of a 32-column chunk, spread over the lanes: lane l holds the
@@ -252,6 +252,57 @@ __device__ __forceinline__ void bias_pack32(float (&y)[32], bool has_bias, const
         y[j + 1] = __fadd_rn(y[j + 1], __uint_as_float(b0 & 0xFFFF0000u));
         y[j + 2] = __fadd_rn(y[j + 2], __uint_as_float(b1 << 16));
         y[j + 3] = __fadd_rn(y[j + 3], __uint_as_float(b1 & 0xFFFF0000u));
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) out[j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
+}
+
+// The same two steps for an output-channel chunk (operands not swapped), with the column
+// constants of columns n0..n0+31 read by every lane from the same addresses (one broadcast
+// load per 4 scales, per 8 biases): fewer instructions than spreading them over the lanes and
+// shuffling. N is a multiple of 8 and w_scale / bias are 16-byte aligned, so each vector load
+// lies wholly inside or wholly past the end of its array (then it is skipped).
+template <bool ASYM>
+__device__ __forceinline__ void dequant32_cols(const Params& p, const uint32_t (&acc)[32], float row_scale,
+                                               int row_int, int64_t n0, float (&y)[32]) {
+  const float e_t = p.w_per_channel ? 0.0f : __ldg(p.w_scale);
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    const int64_t n = n0 + j;
+    const bool in = n < p.cols;
+    float4 e4 = make_float4(e_t, e_t, e_t, e_t);
+    if (p.w_per_channel) e4 = in ? __ldg(reinterpret_cast<const float4*>(p.w_scale + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float e[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float a;
+      if constexpr (ASYM) {
+        const int rs = in ? __ldg(p.w_rowsum + n + u) : 0;
+        const long long t = static_cast<long long>(static_cast<int32_t>(acc[j + u])) -
+                            static_cast<long long>(row_int) * static_cast<long long>(rs);
+        a = __ll2float_rn(t);
+      } else {
+        a = static_cast<float>(static_cast<int32_t>(acc[j + u]));
+      }
+      y[j + u] = __fmul_rn(__fmul_rn(a, row_scale), e[u]);
+    }
+  }
+}
+
+__device__ __forceinline__ void bias_pack32_cols(const Params& p, float (&y)[32], bool has_bias, int64_t n0,
+                                                 uint32_t (&out)[16]) {
+  if (has_bias) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+      const int64_t n = n0 + j;
+      const uint4 b4 = n < p.cols ? __ldg(reinterpret_cast<const uint4*>(p.bias + n)) : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t b[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        y[j + 2 * u] = __fadd_rn(y[j + 2 * u], __uint_as_float(b[u] << 16));
+        y[j + 2 * u + 1] = __fadd_rn(y[j + 2 * u + 1], __uint_as_float(b[u] & 0xFFFF0000u));
       }
     }
   }
@@ -572,7 +623,10 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           if constexpr (ASYM) row_int = __ldg(p.x_zero + r);
         }
       }
-      const ColConsts cc = load_col_consts<SWAP, ASYM>(p, n_half0, lane, kChunks);
+      // swapped operands spread the per-token column constants over the lanes; otherwise
+      // the column constants are broadcast loads inside the chunk loop
+      ColConsts cc{};
+      if constexpr (SWAP) cc = load_col_consts<SWAP, ASYM>(p, n_half0, lane, kChunks);
       const bool has_bias = p.bias != nullptr;
       // lane 0 waits and the warp follows its verdict, so the warp stays converged
       int ok = 0;
@@ -597,7 +651,10 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             tmem_wait_ld();
             const int nvalid = (p.cols - n0) < 32 ? static_cast<int>(p.cols - n0) : 32;
             float y[32];
-            dequant32<SWAP, ASYM>(acc, row_scale, row_int, cc, c, y);
+            if constexpr (SWAP)
+              dequant32<SWAP, ASYM>(acc, row_scale, row_int, cc, c, y);
+            else
+              dequant32_cols<ASYM>(p, acc, row_scale, row_int, n0, y);
             if (p.acc_out != nullptr && r_ok) store_acc32<SWAP>(p, acc, r, n0, nvalid);
             if constexpr (OUTLIERS) {
               if (kb_o > 0) {
@@ -608,7 +665,10 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 for (int j = 0; j < 32; ++j) y[j] = __fadd_rn(y[j], __uint_as_float(of[j]));
               }
             }
-            bias_pack32<SWAP>(y, has_bias, cc, c, row_bias, packed[c]);
+            if constexpr (SWAP)
+              bias_pack32<SWAP>(y, has_bias, cc, c, row_bias, packed[c]);
+            else
+              bias_pack32_cols(p, y, has_bias, n0, packed[c]);
           }
         }
         // the accumulator is no longer needed: hand it back before storing
@@ -687,10 +747,16 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
               }
             }
             float y[32];
-            dequant32<SWAP, ASYM>(acc, row_scale, row_int, cc, c, y);
-            if (p.acc_out != nullptr && r_ok) store_acc32<SWAP>(p, acc, r, n0, nvalid);
             uint32_t packed[16];
-            bias_pack32<SWAP>(y, has_bias, cc, c, row_bias, packed);
+            if constexpr (SWAP) {
+              dequant32<SWAP, ASYM>(acc, row_scale, row_int, cc, c, y);
+              if (p.acc_out != nullptr && r_ok) store_acc32<SWAP>(p, acc, r, n0, nvalid);
+              bias_pack32<SWAP>(y, has_bias, cc, c, row_bias, packed);
+            } else {
+              dequant32_cols<ASYM>(p, acc, row_scale, row_int, n0, y);
+              if (p.acc_out != nullptr && r_ok) store_acc32<SWAP>(p, acc, r, n0, nvalid);
+              bias_pack32_cols(p, y, has_bias, n0, packed);
+            }
             store_box<SWAP>(packed, stage_tiles, ebuf, lane, &tmY, n0, box_row0);
           }
         }

@@ -233,7 +233,12 @@ quant_rows_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
 #pragma unroll
           for (int c = 0; c < CHUNKS; ++c) {
             const int64_t k = c * step + t * 16;
-            if (k < K) store_q16(qrow + k, v[c], r);
+            if (k < K) {
+              if constexpr (MODE == kPerRow)
+                store_q16_own_max(qrow + k, v[c], r);
+              else
+                store_q16(qrow + k, v[c], r);
+            }
           }
         } else {
           for (int64_t k = t * 16; k < K; k += step) {
@@ -249,7 +254,10 @@ quant_rows_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
               }
             }
             finish_chunk<OUTLIERS, HAS_VEC>(rr, row, k, vv, ov, true, w);
-            store_q16(qrow + k, w, r);
+            if constexpr (MODE == kPerRow)
+              store_q16_own_max(qrow + k, w, r);
+            else
+              store_q16(qrow + k, w, r);
           }
         }
         if constexpr (OUTLIERS) {

@@ -9,9 +9,11 @@ namespace rows {
 
 constexpr int kCta = 256;  // minimum CTA size of the row kernels
 
+// The low bytes of a, b, c, d as one little-endian word (three byte permutes).
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
-  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
-         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
+  const uint32_t ab = __byte_perm(static_cast<uint32_t>(a), static_cast<uint32_t>(b), 0x0040u);
+  const uint32_t cd = __byte_perm(static_cast<uint32_t>(c), static_cast<uint32_t>(d), 0x0040u);
+  return __byte_perm(ab, cd, 0x5410u);
 }
 
 // clamp(rne(x * r), -128, 127), returned in the low byte (the upper bytes are not the code).
@@ -50,29 +52,51 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
   return r;
 }
 
-// q8 of two values at once (the products and the rounding add packed; the clamp between them
-// keeps the two from fusing).
+// q8 of two values at once. With CLAMP the products and the rounding add are packed, and
+// the clamp between them keeps the two from fusing. Without CLAMP the caller guarantees
+// |x * r| < 127.5: a row scaled by r = 127/a with a its own absmax (|x| <= a, r finite) stays
+// within 127 * (1 + 2^-24)^2, which rounds to a code in [-127, 127], so the clamp could not
+// change a code; the products are then scalar multiplies with an explicit rounding mode, which
+// are never contracted into the add (a fused multiply-add would round only once).
+template <bool CLAMP>
 __device__ __forceinline__ void q8x2(float x0, float x1, uint64_t r2, int& q0, int& q1) {
   float t0, t1;
-  f2_unpack(f2_mul(f2_pack(x0, x1), r2), t0, t1);
-  t0 = fminf(fmaxf(t0, -128.0f), 127.0f);
-  t1 = fminf(fmaxf(t1, -128.0f), 127.0f);
+  if constexpr (CLAMP) {
+    f2_unpack(f2_mul(f2_pack(x0, x1), r2), t0, t1);
+    t0 = fminf(fmaxf(t0, -128.0f), 127.0f);
+    t1 = fminf(fmaxf(t1, -128.0f), 127.0f);
+  } else {
+    float r, r_hi;
+    f2_unpack(r2, r, r_hi);
+    t0 = __fmul_rn(x0, r);
+    t1 = __fmul_rn(x1, r_hi);
+  }
   f2_unpack(f2_add(f2_pack(t0, t1), f2_pack(12582912.0f, 12582912.0f)), t0, t1);
   q0 = __float_as_int(t0);
   q1 = __float_as_int(t1);
 }
 
+template <bool CLAMP = true>
 __device__ __forceinline__ void store_q16(int8_t* dst, const float (&v)[16], float r) {
   const uint64_t r2 = f2_pack(r, r);
   int q[16];
 #pragma unroll
-  for (int i = 0; i < 16; i += 2) q8x2(v[i], v[i + 1], r2, q[i], q[i + 1]);
+  for (int i = 0; i < 16; i += 2) q8x2<CLAMP>(v[i], v[i + 1], r2, q[i], q[i + 1]);
   uint4 o;
   o.x = pack4(q[0], q[1], q[2], q[3]);
   o.y = pack4(q[4], q[5], q[6], q[7]);
   o.z = pack4(q[8], q[9], q[10], q[11]);
   o.w = pack4(q[12], q[13], q[14], q[15]);
   *reinterpret_cast<uint4*>(dst) = o;
+}
+
+// Codes of 16 values of a row quantized with its own absmax a (r = 127/a): the clamp is
+// needed only when r overflowed to infinity (a < 127 / FLT_MAX), a branch uniform over the row.
+__device__ __forceinline__ void store_q16_own_max(int8_t* dst, const float (&v)[16], float r) {
+  if (r <= 3.402823466e38f)
+    store_q16<false>(dst, v, r);
+  else
+    store_q16<true>(dst, v, r);
 }
 
 // Codes of 16 values with a zero point: clamp(rne(v * r) + z, -128, 127).

@@ -225,7 +225,7 @@ norm_quant_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
 #pragma unroll
       for (int c = 0; c < CHUNKS; ++c) {
         const int64_t k = c * step + t * 16;
-        if (k < K && SQ_GUARD(k + 16 <= K)) store_q16(qrow + k, x[c], r);
+        if (k < K && SQ_GUARD(k + 16 <= K)) store_q16_own_max(qrow + k, x[c], r);
       }
     }
   }

@@ -348,9 +348,13 @@ __device__ __forceinline__ void store_box(const uint32_t (&v)[16], uint8_t* stag
       st[(2 * j + 1) * 32] = static_cast<uint16_t>(v[j] >> 16);
     }
   } else {
+    // the output map uses the 64-byte swizzle: 16-byte granule j of staging row l sits at
+    // granule j ^ ((l >> 1) & 3) (the tile is 2048-byte aligned), so the 32 lanes' stores
+    // spread over all eight 16-byte bank groups (4 wavefronts per instruction, not 16)
     uint4* st = reinterpret_cast<uint4*>(tile + lane * 64);
+    const int sw = (lane >> 1) & 3;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) st[j] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    for (int j = 0; j < 4; ++j) st[j ^ sw] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
   }
   fence_proxy_async_smem();
   __syncwarp();
@@ -900,8 +904,10 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
     *why = "cuTensorMapEncodeTiled failed for the int8 operands";
     return cudaErrorInvalidValue;
   }
+  // 32 x 32 bf16 boxes (64-byte rows); row-major staging is swizzled (see store_box), the
+  // transposed staging of swapped operands is written conflict-free as it is
   if (!make_map(&tmY, a.Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.M),
-                static_cast<uint64_t>(a.N) * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+                static_cast<uint64_t>(a.N) * 2, 32, 32, SWAP ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_64B)) {
     *why = "cuTensorMapEncodeTiled failed for the output";
     return cudaErrorInvalidValue;
   }

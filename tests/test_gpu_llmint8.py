@@ -29,17 +29,20 @@ def test_tiny_config_outliers_are_channels_0_1():
     assert g["count"] == 2 and list(o["idx"]) == [0, 1]
 
 
+# (2433, 1800, 272) runs on CTA pairs (256 x 256 tiles; 70 outlier columns = two bf16 k-blocks)
 @pytest.mark.parametrize("M,N,K,nout", [(5, 24, 48, 1), (130, 72, 144, 3), (200, 264, 208, 7),
                                         (257, 1000, 528, 70), (1024, 2048, 1024, 10), (64, 4096, 4096, 6),
-                                        (300, 9480, 528, 5)])
+                                        (300, 9480, 528, 5), (2433, 1800, 272, 70)])
 def test_random_ragged(M, N, K, nout):
     p = wl.random_problem(M, N, K, seed=M + 3 * N + K, outliers=nout, offset=25.0)
     g, _ = _check(p)
     assert g["count"] == nout
 
 
-def test_no_outliers_is_plain_w8a8():
-    p = wl.random_problem(96, 136, 272, seed=4, outliers=0)
+@pytest.mark.parametrize("M,N,K", [(96, 136, 272), (2433, 1800, 272)])
+def test_no_outliers_is_plain_w8a8(M, N, K):
+    """No outlier column: the kernel double-buffers its int32 accumulator (also on CTA pairs)."""
+    p = wl.random_problem(M, N, K, seed=4, outliers=0)
     g, _ = _check(p, threshold=1e30)
     assert g["count"] == 0
 

@@ -151,72 +151,53 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// Per-warp column constants of a 32-column chunk, spread over the lanes: lane l holds the
-// scales of columns 4*(l%8)..4*(l%8)+3 of chunk l/8 (float4) and their 4 bf16 biases,
-// so a warp covers 4 chunks (128 columns). Loaded before the accumulator is ready.
-// Columns are output channels (weight scale, bias) or, with swapped operands, tokens
-// (per-token activation scale; the bias then belongs to the row).
-struct ColConsts {
-  float4 e;
-  uint2 b;
-  int4 z;  // asymmetric activations: the column's integer factor of the zero-point correction
+// Swapped operands (tokens on the columns): per-warp token constants of a 32-column chunk,
+// spread over the lanes: lane l holds the per-token scales of columns 4*(l%8)..4*(l%8)+3 of
+// chunk l/8 (and their zero points with asymmetric activations), so a warp covers 4 chunks
+// (128 tokens). Loaded before the accumulator is ready. x_scale / x_zero have no alignment
+// contract and M need not be a multiple of 4: scalar loads.
+struct TokenConsts {
+  float4 d;
+  int4 z;  // asymmetric activations: the token's zero point
 };
 
-template <bool SWAP, bool ASYM>
-__device__ __forceinline__ ColConsts load_col_consts(const Params& p, int64_t n_half0, int lane, int chunks) {
-  ColConsts cc;
+template <bool ASYM>
+__device__ __forceinline__ TokenConsts load_token_consts(const Params& p, int64_t n_half0, int lane, int chunks) {
+  TokenConsts tc;
   const int c = lane >> 3;
   const int64_t n = n_half0 + c * 32 + (lane & 7) * 4;
   const bool ok = c < chunks && n < p.cols;
-  cc.z = make_int4(0, 0, 0, 0);
-  if constexpr (SWAP) {
-    // x_scale / x_zero have no alignment contract and M need not be a multiple of 4: scalar loads
-    float v[4];
-    int zz[4];
+  float v[4];
+  int zz[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const bool in = ok && n + i < p.cols;
-      v[i] = in ? __ldg(p.x_scale + (p.x_per_token ? n + i : 0)) : 0.0f;
-      zz[i] = (ASYM && in) ? __ldg(p.x_zero + n + i) : 0;
-    }
-    cc.e = make_float4(v[0], v[1], v[2], v[3]);
-    cc.b = make_uint2(0u, 0u);
-    if constexpr (ASYM) cc.z = make_int4(zz[0], zz[1], zz[2], zz[3]);
-  } else {
-    if constexpr (ASYM) {
-      if (ok) cc.z = make_int4(__ldg(p.w_rowsum + n), __ldg(p.w_rowsum + n + 1), __ldg(p.w_rowsum + n + 2),
-                               __ldg(p.w_rowsum + n + 3));
-    }
-    if (p.w_per_channel) {
-      cc.e = ok ? __ldg(reinterpret_cast<const float4*>(p.w_scale + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
-    } else {
-      const float e0 = __ldg(p.w_scale);
-      cc.e = make_float4(e0, e0, e0, e0);
-    }
-    cc.b = (p.bias != nullptr && ok) ? __ldg(reinterpret_cast<const uint2*>(p.bias + n)) : make_uint2(0u, 0u);
+  for (int i = 0; i < 4; ++i) {
+    const bool in = ok && n + i < p.cols;
+    v[i] = in ? __ldg(p.x_scale + (p.x_per_token ? n + i : 0)) : 0.0f;
+    zz[i] = (ASYM && in) ? __ldg(p.x_zero + n + i) : 0;
   }
-  return cc;
+  tc.d = make_float4(v[0], v[1], v[2], v[3]);
+  tc.z = make_int4(zz[0], zz[1], zz[2], zz[3]);
+  return tc;
 }
 
-// y[j] = (float(acc[j]) * d_m) * e_n for the 32 columns of chunk c: d_m is the row
-// constant and e_n comes from the lanes' column constants, or, with swapped operands,
-// d_m comes from the column constants and e_n is the row constant. With asymmetric
-// activations acc is first corrected in 64-bit integers, acc - z_m * rowsum_n, the row's
-// integer factor times the column's (z_m and rowsum_n, or rowsum_n and z_m if swapped).
-template <bool SWAP, bool ASYM>
-__device__ __forceinline__ void dequant32(const uint32_t (&acc)[32], float row_scale, int row_int,
-                                          const ColConsts& cc, int c, float (&y)[32]) {
+// Swapped operands: y[j] = (float(acc[j]) * d_m) * e_n for the 32 tokens m of chunk c of
+// output channel n (the thread's row): d_m comes from the lanes' token constants (shuffled),
+// e_n is the row constant. With asymmetric activations acc is first corrected in 64-bit
+// integers, acc - z_m * rowsum_n (rowsum_n is the row's integer factor).
+template <bool ASYM>
+__device__ __forceinline__ void dequant32_tokens(const uint32_t (&acc)[32], float row_scale, int row_int,
+                                                 const TokenConsts& tc, int c, float (&y)[32]) {
 #pragma unroll
   for (int j = 0; j < 32; j += 4) {
     const int src = c * 8 + j / 4;
-    const float e[4] = {__shfl_sync(0xffffffffu, cc.e.x, src), __shfl_sync(0xffffffffu, cc.e.y, src),
-                        __shfl_sync(0xffffffffu, cc.e.z, src), __shfl_sync(0xffffffffu, cc.e.w, src)};
+    const float d[4] = {__shfl_sync(0xffffffffu, tc.d.x, src), __shfl_sync(0xffffffffu, tc.d.y, src),
+                        __shfl_sync(0xffffffffu, tc.d.z, src), __shfl_sync(0xffffffffu, tc.d.w, src)};
     int zc[4] = {0, 0, 0, 0};
     if constexpr (ASYM) {
-      zc[0] = __shfl_sync(0xffffffffu, cc.z.x, src);
-      zc[1] = __shfl_sync(0xffffffffu, cc.z.y, src);
-      zc[2] = __shfl_sync(0xffffffffu, cc.z.z, src);
-      zc[3] = __shfl_sync(0xffffffffu, cc.z.w, src);
+      zc[0] = __shfl_sync(0xffffffffu, tc.z.x, src);
+      zc[1] = __shfl_sync(0xffffffffu, tc.z.y, src);
+      zc[2] = __shfl_sync(0xffffffffu, tc.z.z, src);
+      zc[3] = __shfl_sync(0xffffffffu, tc.z.w, src);
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -228,42 +209,30 @@ __device__ __forceinline__ void dequant32(const uint32_t (&acc)[32], float row_s
       } else {
         a = static_cast<float>(static_cast<int32_t>(acc[j + u]));
       }
-      y[j + u] = SWAP ? __fmul_rn(__fmul_rn(a, e[u]), row_scale) : __fmul_rn(__fmul_rn(a, row_scale), e[u]);
+      y[j + u] = __fmul_rn(__fmul_rn(a, d[u]), row_scale);
     }
   }
 }
 
-// y[j] += bias (per column, or the row's bias with swapped operands) when there is one,
-// then pack to bf16 pairs.
-template <bool SWAP>
-__device__ __forceinline__ void bias_pack32(float (&y)[32], bool has_bias, const ColConsts& cc, int c,
-                                            float row_bias, uint32_t (&out)[16]) {
+// Swapped operands: y[j] += the row's (output channel's) bias when there is one, then pack
+// to bf16 pairs.
+__device__ __forceinline__ void bias_pack32_tokens(float (&y)[32], bool has_bias, float row_bias,
+                                                   uint32_t (&out)[16]) {
   if (has_bias) {
-    if constexpr (SWAP) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) y[j] = __fadd_rn(y[j], row_bias);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        const int src = c * 8 + j / 4;
-        const uint32_t b0 = __shfl_sync(0xffffffffu, cc.b.x, src);
-        const uint32_t b1 = __shfl_sync(0xffffffffu, cc.b.y, src);
-        y[j] = __fadd_rn(y[j], __uint_as_float(b0 << 16));
-        y[j + 1] = __fadd_rn(y[j + 1], __uint_as_float(b0 & 0xFFFF0000u));
-        y[j + 2] = __fadd_rn(y[j + 2], __uint_as_float(b1 << 16));
-        y[j + 3] = __fadd_rn(y[j + 3], __uint_as_float(b1 & 0xFFFF0000u));
-      }
-    }
+    for (int j = 0; j < 32; ++j) y[j] = __fadd_rn(y[j], row_bias);
   }
 #pragma unroll
   for (int j = 0; j < 16; ++j) out[j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
 }
 
-// The same two steps for an output-channel chunk (operands not swapped), with the column
-// constants of columns n0..n0+31 read by every lane from the same addresses (one broadcast
-// load per 4 scales, per 8 biases): fewer instructions than spreading them over the lanes and
-// shuffling. N is a multiple of 8 and w_scale / bias are 16-byte aligned, so each vector load
-// lies wholly inside or wholly past the end of its array (then it is skipped).
+// Operands not swapped (output channels on the columns): y[j] = (float(acc[j]) * d_m) * e_n
+// with d_m the row constant, then + bias_n and bf16 packing; the column constants of columns
+// n0..n0+31 are read by every lane from the same addresses (one broadcast load per 4 scales,
+// per 8 biases): fewer instructions than spreading them over the lanes and shuffling. With
+// asymmetric activations acc is first corrected in 64-bit integers, acc - z_m * rowsum_n.
+// N is a multiple of 8 and w_scale / bias are 16-byte aligned, so each vector load lies
+// wholly inside or wholly past the end of its array (then it is skipped).
 template <bool ASYM>
 __device__ __forceinline__ void dequant32_cols(const Params& p, const uint32_t (&acc)[32], float row_scale,
                                                int row_int, int64_t n0, float (&y)[32]) {
@@ -374,7 +343,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                  const __grid_constant__ CUtensorMap tmXo, const __grid_constant__ CUtensorMap tmWo,
                  const __grid_constant__ CUtensorMap tmY, const Params p) {
   using C = Cfg<BN, OUTLIERS, ACC_BUFS, PAIR>;
-  static_assert(!PAIR || (!SWAP && !OUTLIERS && BN == 256), "CTA pairs: plain 256 x 256 tiles");
+  static_assert(!PAIR || (!SWAP && BN == 256), "CTA pairs: 256 x 256 tiles, operands not swapped");
   // rows of A per output tile: one CTA's 128, or a pair's 256 (this CTA's half at rank * 128)
   constexpr int kTileM = PAIR ? 2 * kBM : kBM;
   extern __shared__ uint8_t smem_raw[];
@@ -471,22 +440,22 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           } else {
             uint8_t* sa = stage_base + stage * C::kStageBytes;
             uint8_t* sb = sa + C::kStageA;
+            // int8 k-blocks of Xq / Wq, then bf16 k-blocks of the gathered outlier columns
+            // (64 bf16 = 128 bytes per row: the same stage geometry)
+            const bool body = kb < kb_i8;
+            const CUtensorMap* map_a = body ? &tmA : &tmXo;
+            const CUtensorMap* map_b = body ? &tmB : &tmWo;
+            const int x = body ? kb * kBK : (kb - kb_i8) * (kBK / 2);
             if constexpr (PAIR) {
               // both CTAs' halves complete on the even CTA's barrier, which expects them all
               if (leader) mbar_arrive_expect_tx(full + stage, 2 * C::kStageBytes);
               const uint32_t fb = mapa_shared(full + stage, 0);
-              tma_load_2d_pair(sa, &tmA, fb, kb * kBK, m0, kEvictNormal);
-              tma_load_2d_pair(sb, &tmB, fb, kb * kBK, n0, kEvictNormal);
+              tma_load_2d_pair(sa, map_a, fb, x, m0, kEvictNormal);
+              tma_load_2d_pair(sb, map_b, fb, x, n0, kEvictNormal);
             } else {
               mbar_arrive_expect_tx(full + stage, C::kStageBytes);
-              if (kb < kb_i8) {
-                tma_load_2d(sa, &tmA, full + stage, kb * kBK, m0, kEvictNormal);
-                tma_load_2d(sb, &tmB, full + stage, kb * kBK, n0, kEvictNormal);
-              } else {
-                const int ko = (kb - kb_i8) * (kBK / 2);
-                tma_load_2d(sa, &tmXo, full + stage, ko, m0, kEvictNormal);
-                tma_load_2d(sb, &tmWo, full + stage, ko, n0, kEvictNormal);
-              }
+              tma_load_2d(sa, map_a, full + stage, x, m0, kEvictNormal);
+              tma_load_2d(sb, map_b, full + stage, x, n0, kEvictNormal);
             }
             issued_mask |= 1u << stage;
             issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -511,7 +480,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && leader) {
       constexpr uint32_t kIdescI8 = idesc_i8_s32(kTileM, BN);
-      constexpr uint32_t kIdescBf16 = idesc_bf16_f32(kBM, BN);
+      constexpr uint32_t kIdescBf16 = idesc_bf16_f32(kTileM, BN);
       // a pair's commits go to the barrier in each CTA (shared::cluster addresses)
       const uint32_t empty_c0 = PAIR ? mapa_shared(empty, 0) : 0u, empty_c1 = PAIR ? mapa_shared(empty, 1) : 0u;
       const uint32_t tfull_c0 = PAIR ? mapa_shared(tmem_full, 0) : 0u;
@@ -542,26 +511,32 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           tc_fence_after();
           const uint32_t a_addr = smem_u32(stage_base + stage * C::kStageBytes);
           const uint32_t b_addr = a_addr + C::kStageA;
-          if constexpr (PAIR) {
+          if (kb < kb_i8) {
 #pragma unroll
-            for (int k = 0; k < kBK / 32; ++k)
-              mma_i8_pair(d_i32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescI8,
-                          (kb != kb0 || k != 0) ? 1u : 0u);
-            mma_commit_pair(empty_c0 + 8u * stage);
-            mma_commit_pair(empty_c1 + 8u * stage);
-          } else if (kb < kb_i8) {
-#pragma unroll
-            for (int k = 0; k < kBK / 32; ++k)
-              mma_i8(d_i32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescI8,
-                     (kb != kb0 || k != 0) ? 1u : 0u);
+            for (int k = 0; k < kBK / 32; ++k) {
+              const uint32_t acc = (kb != kb0 || k != 0) ? 1u : 0u;
+              if constexpr (PAIR)
+                mma_i8_pair(d_i32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescI8, acc);
+              else
+                mma_i8(d_i32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescI8, acc);
+            }
           } else {
             const int ko = kb - kb_i8;
 #pragma unroll
-            for (int k = 0; k < kBK / 32; ++k)
-              mma_f16(d_f32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescBf16,
-                      (ko | k) != 0);
+            for (int k = 0; k < kBK / 32; ++k) {
+              const uint32_t acc = (ko | k) != 0 ? 1u : 0u;
+              if constexpr (PAIR)
+                mma_f16_pair(d_f32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescBf16, acc);
+              else
+                mma_f16(d_f32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescBf16, acc);
+            }
           }
-          if constexpr (!PAIR) mma_commit(empty + stage);
+          if constexpr (PAIR) {
+            mma_commit_pair(empty_c0 + 8u * stage);
+            mma_commit_pair(empty_c1 + 8u * stage);
+          } else {
+            mma_commit(empty + stage);
+          }
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1;
@@ -629,8 +604,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       }
       // swapped operands spread the per-token column constants over the lanes; otherwise
       // the column constants are broadcast loads inside the chunk loop
-      ColConsts cc{};
-      if constexpr (SWAP) cc = load_col_consts<SWAP, ASYM>(p, n_half0, lane, kChunks);
+      TokenConsts tc{};
+      if constexpr (SWAP) tc = load_token_consts<ASYM>(p, n_half0, lane, kChunks);
       const bool has_bias = p.bias != nullptr;
       // lane 0 waits and the warp follows its verdict, so the warp stays converged
       int ok = 0;
@@ -656,7 +631,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             const int nvalid = (p.cols - n0) < 32 ? static_cast<int>(p.cols - n0) : 32;
             float y[32];
             if constexpr (SWAP)
-              dequant32<SWAP, ASYM>(acc, row_scale, row_int, cc, c, y);
+              dequant32_tokens<ASYM>(acc, row_scale, row_int, tc, c, y);
             else
               dequant32_cols<ASYM>(p, acc, row_scale, row_int, n0, y);
             if (p.acc_out != nullptr && r_ok) store_acc32<SWAP>(p, acc, r, n0, nvalid);
@@ -670,7 +645,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
               }
             }
             if constexpr (SWAP)
-              bias_pack32<SWAP>(y, has_bias, cc, c, row_bias, packed[c]);
+              bias_pack32_tokens(y, has_bias, row_bias, packed[c]);
             else
               bias_pack32_cols(p, y, has_bias, n0, packed[c]);
           }
@@ -753,9 +728,9 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             float y[32];
             uint32_t packed[16];
             if constexpr (SWAP) {
-              dequant32<SWAP, ASYM>(acc, row_scale, row_int, cc, c, y);
+              dequant32_tokens<ASYM>(acc, row_scale, row_int, tc, c, y);
               if (p.acc_out != nullptr && r_ok) store_acc32<SWAP>(p, acc, r, n0, nvalid);
-              bias_pack32<SWAP>(y, has_bias, cc, c, row_bias, packed);
+              bias_pack32_tokens(y, has_bias, row_bias, packed);
             } else {
               dequant32_cols<ASYM>(p, acc, row_scale, row_int, n0, y);
               if (p.acc_out != nullptr && r_ok) store_acc32<SWAP>(p, acc, r, n0, nvalid);
@@ -865,7 +840,7 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool outliers) {
     pl.bn = 256;
     // CTA pairs when the 256 x 256 tiles still give every pair of SMs a tile
     const int64_t pair_tiles = ((rows + 2 * kBM - 1) / (2 * kBM)) * ((cols + 255) / 256);
-    if (!outliers && pair_tiles >= kPlanSms / 2) {
+    if (pair_tiles >= kPlanSms / 2) {
       pl.pair = true;
       pl.num_full = static_cast<int>(pair_tiles);
       return pl;
@@ -914,7 +889,7 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   if (OUTLIERS) {
     const uint64_t ldo = static_cast<uint64_t>(a.ld_o);
     if (!make_operand_map(&tmXo, a.Xo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ldo, a.M, ldo * 2, kBM) ||
-        !make_operand_map(&tmWo, a.Wo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ldo, a.N, ldo * 2, BN)) {
+        !make_operand_map(&tmWo, a.Wo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ldo, a.N, ldo * 2, PAIR ? BN / 2 : BN)) {
       *why = "cuTensorMapEncodeTiled failed for the outlier operands";
       return cudaErrorInvalidValue;
     }
@@ -992,6 +967,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream, const char** why
   const Plan pl = plan_gemm(a.M, a.N, a.K, outliers);
   if (outliers) {
     // int32 + fp32 accumulators: 256-wide tiles fit TMEM once, narrower ones twice
+    if (pl.pair) return run<256, true, 1, false, false, true>(a, pl, stream, why);
     if (pl.bn == 256) return run<256, true, 1, false>(a, pl, stream, why);
     if (pl.bn == 128) return run<128, true, 2, false>(a, pl, stream, why);
     return run<64, true, 2, false>(a, pl, stream, why);

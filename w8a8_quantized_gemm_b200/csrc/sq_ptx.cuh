@@ -292,6 +292,17 @@ __device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// Pair MMA, bf16 x bf16 -> fp32 (issued by the even CTA only).
+__device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // The mbarrier at `cluster_addr` (this CTA's or the peer's) tracks completion of all prior
 // pair MMAs issued by this thread.
 __device__ __forceinline__ void mma_commit_pair(uint32_t cluster_addr) {

@@ -41,8 +41,8 @@ N_SETS = 4  # rotating input sets: 4 x (16.8 MB X + 90.2 MB W) = 428 MB > 126 MB
 # DRAM traffic of one int8 GEMM launch on this workload (dram__bytes_read.sum +
 # dram__bytes_write.sum of an ncu capture of `python -m w8a8_quantized_gemm_b200.profile_cases
 # gemm`), valid while the GEMM source's code (comments aside) hashes to GEMM_SRC_SHA.
-NCU_GEMM_TRAFFIC_BYTES = 53596928 + 13813504
-GEMM_SRC_SHA = "2fe704e4a1e2e742"
+NCU_GEMM_TRAFFIC_BYTES = 53596928 + 13500928
+GEMM_SRC_SHA = "475f5f6624991864"
 
 
 def _peaks():

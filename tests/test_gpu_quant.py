@@ -85,6 +85,27 @@ def test_quant_act_zero_rows_and_ties():
     assert np.all(q[[0, 1, 3, 4]] == 0) and np.all(host(d)[[0, 1, 3, 4]] == 0)
 
 
+@pytest.mark.parametrize("K", [272, 8192])
+def test_quant_act_tiny_row_absmax(K):
+    """Rows of tiny magnitude: below an absmax of 127 / FLT_MAX (about 3.7e-37) the factor
+    127/a overflows to infinity on both sides and every code saturates to 127 or -128 (the
+    kernel's clamped branch); just above it the factor is finite and near FLT_MAX (the
+    unclamped branch). Non-zero values only: 0 * inf has no code."""
+    rng = np.random.default_rng(K)
+    M = 4
+    x = rng.uniform(0.5, 2.0, (M, K)).astype(np.float32) * np.where(rng.random((M, K)) < 0.5, -1.0, 1.0)
+    x[0] *= np.float32(1e-37)     # absmax ~2e-37: 127/a = inf
+    x[2] *= np.float32(2.2e-37)   # absmax ~4.4e-37: 127/a ~ 2.9e38, finite
+    X = wl.f32_to_bf16_bits(x.astype(np.float32))
+    Xq, d = empty((M, K), torch.int8), empty(M, torch.float32)
+    sq.sq_quant_act_per_token(dev_bf16(X), None, Xq, d)
+    oq, od = oracle.quant_act_per_token(X, None)
+    assert np.array_equal(host(Xq), oq)
+    assert np.array_equal(host(d), od)
+    assert set(np.unique(oq[0]).tolist()) <= {127, -128}
+    assert np.abs(oq[2].astype(np.int32)).max() == 127 and np.unique(oq[2]).size > 2
+
+
 @pytest.mark.parametrize("gran", [sq.SQ_PER_CHANNEL, sq.SQ_PER_TENSOR])
 @pytest.mark.parametrize("N,K", [(1, 16), (13, 528), (256, 256), (300, 4096), (64, 8208), (8, 20000)])
 def test_smooth_quant_weight_exact(gran, N, K):

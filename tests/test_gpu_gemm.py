@@ -33,11 +33,13 @@ def _gemm_direct(xq, wq, d, e, gran, bias_bits):
 # fills the SMs with whole swapped tiles, (1,4096,4096) splits them, (65,296,512) does not swap;
 # (2304,2120,720), (2433,1800,272) and (4100,1288,1040) run on CTA pairs (256 x 256 tiles): the
 # last column tile leaves the odd CTA's half of B out of range, 2433 and 4100 leave the odd
-# CTA's rows of the last row tile (nearly) empty, 4100 x 1288 takes two passes of the pairs
+# CTA's rows of the last row tile (nearly) empty, 4100 x 1288 takes two passes of the pairs;
+# (100, 37888, 128) fills the SMs with 256-wide tiles of one 128-row tile (no pairs: the odd
+# CTA would only compute padding)
 GEMM_SHAPES = [(1, 8, 16), (16, 256, 256), (5, 24, 48), (130, 72, 144), (200, 264, 208), (128, 128, 4096),
                (257, 1000, 528), (3, 200, 1040), (64, 4096, 4096), (1024, 2048, 1024), (300, 9480, 528),
                (2304, 2120, 720), (37, 9736, 256), (1, 4096, 4096), (65, 296, 512), (2433, 1800, 272),
-               (4100, 1288, 1040)]
+               (4100, 1288, 1040), (100, 37888, 128)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)

@@ -820,12 +820,13 @@ constexpr int64_t kSwapMaxM = 64;  // token counts that fit one 64-column tile
 // Operand roles: up to 64 tokens (and no outlier product) swap the operands, so the weight
 // rows fill the 128-row MMA operand and the tokens one 64-column tile. Otherwise the tile
 // width is the widest of 256/128/64 whose tile count covers the SMs; 256-wide tiles become
-// 256 x 256 CTA-pair tiles when those still cover the SM pairs (each CTA then stages
-// two thirds of the bytes per k-block of a one-CTA 128 x 256 tile). Problems with fewer
-// tiles than half the SMs (small M, or a swapped decode shape) split every tile along K
-// into S parts whose exact int32 partials meet in the workspace. (Splitting only the tiles
-// of a last partial wave was measured slower on the 2048 x 11008 x 4096 shape, so whole
-// tiles are kept there.) LLM.int8 (outlier operands) tiles are never split.
+// 256 x 256 CTA-pair tiles when those still cover the SM pairs without padding rows (each
+// CTA then stages two thirds of the bytes per k-block of a one-CTA 128 x 256 tile).
+// Problems with fewer tiles than half the SMs (small M, or a swapped decode shape) split
+// every tile along K into S parts whose exact int32 partials meet in the workspace.
+// (Splitting only the tiles of a last partial wave was measured slower on the
+// 2048 x 11008 x 4096 shape, so whole tiles are kept there.) LLM.int8 (outlier operands)
+// tiles are never split.
 Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool outliers) {
   const bool swap = !outliers && M <= kSwapMaxM;
   const int64_t rows = swap ? N : M;
@@ -838,9 +839,12 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool outliers) {
     pl.bn = 64;
   } else if (tiles(256) >= kPlanSms) {
     pl.bn = 256;
-    // CTA pairs when the 256 x 256 tiles still give every pair of SMs a tile
+    // CTA pairs when the 256 x 256 tiles still give every pair of SMs a tile and add no
+    // padded rows (an even number of 128-row tiles) or few (at least 32 of them): with
+    // 65..128 rows, say, the odd CTA of every pair would only compute padding
     const int64_t pair_tiles = ((rows + 2 * kBM - 1) / (2 * kBM)) * ((cols + 255) / 256);
-    if (pair_tiles >= kPlanSms / 2) {
+    const bool pair_rows = m_t % 2 == 0 || m_t >= 32;
+    if (pair_rows && pair_tiles >= kPlanSms / 2) {
       pl.pair = true;
       pl.num_full = static_cast<int>(pair_tiles);
       return pl;

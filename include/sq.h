@@ -359,6 +359,17 @@ SQ_API uint64_t sq_kernel_launch_count(void);
  * use; the output of the armed call is undefined. */
 SQ_API void sq_debug_arm_fault(int fault, uint64_t wait_limit_ns);
 
+/* Test hook (no counterpart on the pages): the launch plan that sq_int8_gemm_dequant
+ * (outliers = 0) or the GEMM of llmint8_decomposed_linear (outliers = 1) uses for an
+ * M x N x K product, computed on the host without touching a device. plan (caller-owned,
+ * 7 entries) receives: [0] path (0 = the CUDA-core product for a few tokens, 1 = tensor
+ * cores with one CTA per output tile, 2 = tensor cores with CTA pairs on 256-row tiles),
+ * [1] 1 if the operands are swapped (weight rows on the 128-row MMA operand), [2] the tile
+ * width BN, [3] whole-tile work units, [4] tiles split along K, [5] parts per split tile,
+ * [6] k-blocks (128 bytes of K) per part. Returns SQ_ERR_INVALID (plan untouched) when a
+ * size is not positive or plan is NULL. */
+SQ_API sq_status sq_debug_gemm_plan(int64_t M, int64_t N, int64_t K, int outliers, int64_t* plan);
+
 #ifdef __cplusplus
 }
 #endif

@@ -542,4 +542,11 @@ void sq_debug_arm_fault(int fault, uint64_t wait_limit_ns) {
   g_arm_limit_ns = wait_limit_ns == 0 ? sq::kDefaultWaitLimitNs : wait_limit_ns;
 }
 
+sq_status sq_debug_gemm_plan(int64_t M, int64_t N, int64_t K, int outliers, int64_t* plan) {
+  if (plan == nullptr || M <= 0 || N <= 0 || K <= 0)
+    return fail(SQ_ERR_INVALID, "sq_debug_gemm_plan: sizes must be positive and plan non-NULL");
+  sq::gemm_plan_numbers(M, N, K, outliers != 0, plan);
+  return SQ_OK;
+}
+
 }  // extern "C"

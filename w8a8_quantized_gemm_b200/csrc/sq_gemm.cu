@@ -964,6 +964,19 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, bool outliers) {
          up256(sizeof(int32_t) * pl.tail_tiles * kEpiWarps);
 }
 
+void gemm_plan_numbers(int64_t M, int64_t N, int64_t K, bool outliers, int64_t* out) {
+  if (gemv_applies(M, K, outliers)) {
+    const int64_t kb = (K + kBK - 1) / kBK;
+    const int64_t v[7] = {0, 0, 0, 0, 0, 1, kb};
+    for (int i = 0; i < 7; ++i) out[i] = v[i];
+    return;
+  }
+  const Plan pl = plan_gemm(M, N, K, outliers);
+  const int64_t v[7] = {pl.pair ? 2 : 1, pl.swap ? 1 : 0, pl.bn, pl.num_full, pl.tail_tiles, pl.splits,
+                        pl.kb_per_split};
+  for (int i = 0; i < 7; ++i) out[i] = v[i];
+}
+
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream, const char** why) {
   const bool outliers = a.Xo != nullptr;
   // up to 4 tokens: a weight stream on the CUDA cores (no tensor-core set-up, no K split)

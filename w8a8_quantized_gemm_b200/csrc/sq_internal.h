@@ -178,6 +178,8 @@ struct GemmArgs {
   int fault = 0;                    // test hook: 1 = producer withholds one stage
 };
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, bool outliers);
+// The launch plan of launch_gemm as 7 numbers (see sq_debug_gemm_plan).
+void gemm_plan_numbers(int64_t M, int64_t N, int64_t K, bool outliers, int64_t* out);
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream, const char** why);
 
 // ---- CUDA-core product for M <= 4 tokens (sq_gemv.cu): same arguments and results as the GEMM.

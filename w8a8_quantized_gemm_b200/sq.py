@@ -53,6 +53,7 @@ _SIGS = {
     "sq_sync_status": ([_p], _i32),
     "sq_version": ([], C.c_char_p),
     "sq_debug_arm_fault": ([_i32, C.c_uint64], None),
+    "sq_debug_gemm_plan": ([_i64, _i64, _i64, _i32, _p], _i32),
     "sq_kernel_launch_count": ([], C.c_uint64),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -311,6 +312,17 @@ def sq_kernel_launch_count() -> int:
 
 def sq_debug_arm_fault(fault: int, wait_limit_ns: int = 0):
     _lib.sq_debug_arm_fault(int(fault), int(wait_limit_ns))
+
+
+GEMM_PLAN_FIELDS = ("path", "swap", "bn", "whole_tiles", "split_tiles", "splits", "kb_per_split")
+GEMM_PATH_CUDA_CORES, GEMM_PATH_TENSOR, GEMM_PATH_TENSOR_PAIRS = 0, 1, 2
+
+
+def sq_debug_gemm_plan(M: int, N: int, K: int, outliers: bool = False) -> dict:
+    """The launch plan of the GEMM for an M x N x K product (host only, no device)."""
+    out = (C.c_int64 * 7)()
+    _check(_lib.sq_debug_gemm_plan(int(M), int(N), int(K), 1 if outliers else 0, C.cast(out, C.c_void_p)))
+    return dict(zip(GEMM_PLAN_FIELDS, (int(v) for v in out)))
 
 
 def workspace(op: int, M: int, N: int, K: int, device="cuda"):

@@ -24,6 +24,10 @@
 // operand (output channels on TMEM lanes) and the tokens the N dimension, so no MMA row
 // and no weight byte is spent on padding; the epilogue then applies the per-token scale
 // per column and the per-channel scale and bias per row, and stores transposed boxes.
+// Large shapes run on CTA pairs (clusters of 2): each pair computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 issued by the even CTA; each CTA stages its own 128 rows of A
+// and 128 rows of B, the loads of both CTAs complete on the even CTA's barriers, and each
+// CTA's epilogue drains its own 128 accumulator rows.
 // Every mbarrier wait is bounded; on timeout the kernel records an error bit in the
 // device status word, drains its own TMA loads and MMAs, frees TMEM and returns.
 #include "sq_internal.h"

@@ -5,10 +5,10 @@ Usage: python -m w8a8_quantized_gemm_b200.profile_cases
 
 Each case makes random device inputs of one workload's shape and calls one entry point three
 times (so that a capture can skip the first, cold launch):
-  gemm    sq_int8_gemm_dequant, 2048 x 11008 x 4096 (Llama-2-7B MLP up-projection)
+  gemm    sq_int8_gemm_dequant, 2048 x 11008 x 4096 (Llama-2-7B MLP up-projection; CTA pairs)
   decode  sq_int8_gemm_dequant, 64 x 4096 x 4096 (decode: swapped operands, split K)
   decode1 sq_int8_gemm_dequant, 1 x 4096 x 4096 (one token: the CUDA-core product)
-  llm     llmint8_decomposed_linear, 2048 x 11008 x 4096 with 4 outlier columns
+  llm     llmint8_decomposed_linear, 2048 x 11008 x 4096 with 4 outlier columns (CTA pairs)
   quant   sq_quant_act_per_token with smoothing, X bf16 [8192, 8192] (inputs larger than L2)
   absmax  sq_act_channel_absmax, X bf16 [8192, 8192]
   norm    sq_norm_smooth_quant (LayerNorm with beta, smoothing), X bf16 [8192, 8192]

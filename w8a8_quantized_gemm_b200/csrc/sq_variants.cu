@@ -319,7 +319,11 @@ finish_threshold_kernel(const double* __restrict__ part1, const double* __restri
 constexpr int kBins = 1 << 15;  // bf16 magnitudes (sign dropped)
 constexpr int kHistThreads = 1024;
 
-// Per-CTA histogram of |x| bit patterns in shared memory, added into the global one.
+// Per-CTA histogram of |x| bit patterns in shared memory, added into the global one. Each
+// thread keeps kHistUnroll 16-byte loads in flight before their shared-memory atomics (one
+// load per thread left the pass short of bytes in flight).
+constexpr int kHistUnroll = 4;
+
 __global__ void __launch_bounds__(kHistThreads)
 abs_hist_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
                 unsigned long long* __restrict__ hist) {
@@ -330,16 +334,29 @@ abs_hist_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64
   __syncthreads();
   const int64_t vecs_per_row = K / 8;
   const int64_t total = rows * vecs_per_row;
-  for (int64_t v = static_cast<int64_t>(blockIdx.x) * kHistThreads + threadIdx.x; v < total;
-       v += static_cast<int64_t>(gridDim.x) * kHistThreads) {
-    const int64_t r = v / vecs_per_row;
-    const int64_t c = v - r * vecs_per_row;
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + r * ld) + c);
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kHistThreads;
+  for (int64_t v0 = static_cast<int64_t>(blockIdx.x) * kHistThreads + threadIdx.x; v0 < total;
+       v0 += stride * kHistUnroll) {
+    uint4 w[kHistUnroll];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      atomicAdd(&sh[u[i] & 0x7FFFu], 1u);
-      atomicAdd(&sh[(u[i] >> 16) & 0x7FFFu], 1u);
+    for (int u = 0; u < kHistUnroll; ++u) {
+      const int64_t v = v0 + u * stride;
+      if (v < total) {
+        const int64_t r = v / vecs_per_row;
+        const int64_t c = v - r * vecs_per_row;
+        w[u] = __ldg(reinterpret_cast<const uint4*>(src + r * ld) + c);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kHistUnroll; ++u) {
+      if (v0 + u * stride < total) {
+        const uint32_t q[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          atomicAdd(&sh[q[i] & 0x7FFFu], 1u);
+          atomicAdd(&sh[(q[i] >> 16) & 0x7FFFu], 1u);
+        }
+      }
     }
   }
   __syncthreads();
@@ -347,37 +364,44 @@ abs_hist_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64
     if (sh[b] != 0u) atomicAdd(hist + b, static_cast<unsigned long long>(sh[b]));
 }
 
-// One CTA of 1024 threads, 32 bins each: the bin holding the element of 1-based rank `rank`
-// (the first bin whose inclusive cumulative count reaches it) gives the value.
+// One CTA of 32 warps; warp w owns the 1024 consecutive bins [1024 w, 1024 w + 1024). The
+// warps' totals (coalesced reads) locate the warp whose bins hold the element of 1-based rank
+// `rank`; that warp walks its bins 32 at a time with an inclusive warp scan and the first bin
+// whose cumulative count reaches the rank gives the value (the bin is the value's bit pattern).
 __global__ void __launch_bounds__(kHistThreads)
 select_rank_kernel(const unsigned long long* __restrict__ hist, unsigned long long rank, float* __restrict__ out) {
   griddep_wait();
   griddep_launch_dependents();
-  constexpr int kPer = kBins / kHistThreads;
-  __shared__ unsigned long long part[kHistThreads];
-  const int t = threadIdx.x;
-  unsigned long long mine = 0;
-#pragma unroll 4
-  for (int i = 0; i < kPer; ++i) mine += hist[t * kPer + i];
-  part[t] = mine;
+  constexpr int kWarps = kHistThreads / 32;
+  constexpr int kPerWarp = kBins / kWarps;
+  __shared__ unsigned long long wsum[kWarps];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const unsigned long long* h = hist + static_cast<int64_t>(warp) * kPerWarp;
+  unsigned long long s = 0;
+  for (int i = lane; i < kPerWarp; i += 32) s += h[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) wsum[warp] = s;
   __syncthreads();
-  // inclusive scan over the 1024 partial counts (Hillis-Steele, exact integers)
-  for (int o = 1; o < kHistThreads; o <<= 1) {
-    const unsigned long long add = t >= o ? part[t - o] : 0ull;
-    __syncthreads();
-    part[t] += add;
-    __syncthreads();
-  }
-  const unsigned long long before = t > 0 ? part[t - 1] : 0ull;
-  if (before < rank && part[t] >= rank) {
-    unsigned long long run = before;
-    for (int i = 0; i < kPer; ++i) {
-      run += hist[t * kPer + i];
-      if (run >= rank && SQ_GUARD(t * kPer + i < kBins)) {
-        *out = __uint_as_float(static_cast<uint32_t>(t * kPer + i) << 16);
-        break;
-      }
+  unsigned long long run = 0;  // count in the bins before this warp's
+  for (int w = 0; w < warp; ++w) run += wsum[w];
+  if (!(run < rank && run + wsum[warp] >= rank)) return;  // warp-uniform
+  for (int i0 = 0; i0 < kPerWarp; i0 += 32) {
+    unsigned long long inc = h[i0 + lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
     }
+    const unsigned hit = __ballot_sync(0xffffffffu, run + inc >= rank);
+    if (hit != 0u) {
+      const int first = __ffs(hit) - 1;
+      const int bin = warp * kPerWarp + i0 + first;
+      if (lane == first && SQ_GUARD(bin < kBins)) *out = __uint_as_float(static_cast<uint32_t>(bin) << 16);
+      break;
+    }
+    run += __shfl_sync(0xffffffffu, inc, 31);
   }
 }
 

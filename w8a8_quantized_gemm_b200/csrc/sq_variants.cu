@@ -252,9 +252,11 @@ cudaError_t launch_norm_t(const uint16_t* src, int64_t rows, int64_t K, int64_t 
 
 // ------------------------------------------------------------------ mean / std threshold
 constexpr int kStatThreads = 256;
+constexpr int kStatUnroll = 4;
 
 // part1[b], part2[b] = sum and sum of squares of the elements of CTA b's rows (fp64, four
-// independent chains per thread, then a fixed-order CTA reduction).
+// independent chains per thread, then a fixed-order CTA reduction). Each thread keeps
+// kStatUnroll 16-byte loads in flight ahead of the conversions and sums.
 __global__ void __launch_bounds__(kStatThreads)
 sum_partials_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int64_t rows_per_cta,
                     double* __restrict__ part1, double* __restrict__ part2) {
@@ -267,17 +269,25 @@ sum_partials_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, i
   double s1a = 0.0, s1b = 0.0, s2a = 0.0, s2b = 0.0;
   for (int64_t r = r0; r < r1; ++r) {
     const uint4* p = reinterpret_cast<const uint4*>(src + r * ld);
-    for (int64_t v = threadIdx.x; v < vecs; v += kStatThreads) {
-      const uint4 w = __ldg(p + v);
-      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+    for (int64_t v0 = threadIdx.x; v0 < vecs; v0 += kStatThreads * kStatUnroll) {
+      uint4 w[kStatUnroll];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const double lo = static_cast<double>(__uint_as_float(u[i] << 16));
-        const double hi = static_cast<double>(__uint_as_float(u[i] & 0xFFFF0000u));
-        s1a = __dadd_rn(s1a, lo);
-        s1b = __dadd_rn(s1b, hi);
-        s2a = __fma_rn(lo, lo, s2a);
-        s2b = __fma_rn(hi, hi, s2b);
+      for (int j = 0; j < kStatUnroll; ++j) {
+        const int64_t v = v0 + j * kStatThreads;
+        w[j] = v < vecs ? __ldg(p + v) : make_uint4(0u, 0u, 0u, 0u);  // zeros add nothing
+      }
+#pragma unroll
+      for (int j = 0; j < kStatUnroll; ++j) {
+        const uint32_t u[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const double lo = static_cast<double>(__uint_as_float(u[i] << 16));
+          const double hi = static_cast<double>(__uint_as_float(u[i] & 0xFFFF0000u));
+          s1a = __dadd_rn(s1a, lo);
+          s1b = __dadd_rn(s1b, hi);
+          s2a = __fma_rn(lo, lo, s2a);
+          s2b = __fma_rn(hi, hi, s2b);
+        }
       }
     }
   }

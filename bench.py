@@ -42,7 +42,7 @@ N_SETS = 4  # rotating input sets: 4 x (16.8 MB X + 90.2 MB W) = 428 MB > 126 MB
 # dram__bytes_write.sum of an ncu capture of `python -m w8a8_quantized_gemm_b200.profile_cases
 # gemm`), valid while the GEMM source's code (comments aside) hashes to GEMM_SRC_SHA.
 NCU_GEMM_TRAFFIC_BYTES = 53596928 + 13500928
-GEMM_SRC_SHA = "e03f80f6b7cca9f2"
+GEMM_SRC_SHA = "3f0e8e578675aa01"
 
 
 def _peaks():

@@ -246,7 +246,8 @@ __device__ __forceinline__ void dequant32_cols(const Params& p, const uint32_t (
     const int64_t n = n0 + j;
     const bool in = n < p.cols;
     float4 e4 = make_float4(e_t, e_t, e_t, e_t);
-    if (p.w_per_channel) e4 = in ? __ldg(reinterpret_cast<const float4*>(p.w_scale + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (p.w_per_channel)
+      e4 = in ? __ldg(reinterpret_cast<const float4*>(p.w_scale + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
     const float e[4] = {e4.x, e4.y, e4.z, e4.w};
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -889,8 +890,9 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   }
   // 32 x 32 bf16 boxes (64-byte rows); row-major staging is swizzled (see store_box), the
   // transposed staging of swapped operands is written conflict-free as it is
+  const CUtensorMapSwizzle y_swizzle = SWAP ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_64B;
   if (!make_map(&tmY, a.Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.M),
-                static_cast<uint64_t>(a.N) * 2, 32, 32, SWAP ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_64B)) {
+                static_cast<uint64_t>(a.N) * 2, 32, 32, y_swizzle)) {
     *why = "cuTensorMapEncodeTiled failed for the output";
     return cudaErrorInvalidValue;
   }

@@ -53,6 +53,23 @@ def test_per_tensor_outlier_example(golden_dir):
     assert q[:, ch].min() == -127 and q[:, ch].max() == 127
 
 
+def test_tiny_absmax_saturates_and_just_above_does_not():
+    """Degenerate rows: an absmax below 127/FLT_MAX makes the fp32 factor 127/a infinite, so
+    the non-zero values saturate (127 or -128); an absmax just above keeps codes in [-127, 127]
+    with both ends reached (the value at the absmax itself maps to exactly +-127)."""
+    x = np.array([[1e-37, -2e-37, 0.5e-37, -1.5e-37],
+                  [4.4e-37, -4.4e-37, 2.2e-37, -1.1e-37]], np.float32)
+    bits = wl.f32_to_bf16_bits(x)
+    xb = _f32(bits)
+    a = np.abs(xb).max(axis=1)
+    with np.errstate(over="ignore"):
+        assert np.isinf(np.float32(127.0) / a[0]) and np.isfinite(np.float32(127.0) / a[1])
+    q, d = oracle.quant_act_per_token(bits, None)
+    assert list(q[0]) == [127, -128, 127, -128]
+    assert q[1].max() == 127 and q[1].min() == -127 and abs(int(q[1, 2])) in (63, 64)
+    assert d[0] == np.float32(a[0] / np.float32(127.0))
+
+
 def test_hand_quantization(golden_dir):
     """量化基础与INT8 quantization-flow example, worked by hand (ties to even)."""
     g = _load(golden_dir, "basics_hand_quant.json")

@@ -29,10 +29,14 @@ def test_tiny_config_outliers_are_channels_0_1():
     assert g["count"] == 2 and list(o["idx"]) == [0, 1]
 
 
-# (2433, 1800, 272) runs on CTA pairs (256 x 256 tiles; 70 outlier columns = two bf16 k-blocks)
+# (2433, 1800, 272) runs on CTA pairs (256 x 256 tiles; 70 outlier columns = two bf16 k-blocks);
+# (2048, 7168, 1152) gives each pair three or four tiles and (384, 32768, 1152) each single CTA
+# two or three (both accumulator buffers reused; nine k-blocks, so each tile's outlier
+# k-blocks run after eight k-blocks of the next tile), (1152, 2304, 256) runs 128-wide tiles
 @pytest.mark.parametrize("M,N,K,nout", [(5, 24, 48, 1), (130, 72, 144, 3), (200, 264, 208, 7),
                                         (257, 1000, 528, 70), (1024, 2048, 1024, 10), (64, 4096, 4096, 6),
-                                        (300, 9480, 528, 5), (2433, 1800, 272, 70)])
+                                        (300, 9480, 528, 5), (2433, 1800, 272, 70), (2048, 7168, 1152, 12),
+                                        (384, 32768, 1152, 12), (1152, 2304, 256, 9)])
 def test_random_ragged(M, N, K, nout):
     p = wl.random_problem(M, N, K, seed=M + 3 * N + K, outliers=nout, offset=25.0)
     g, _ = _check(p)

@@ -266,13 +266,16 @@ def test_three_sigma_example_through_llmint8():
     Wq, e = empty((N, K), torch.int8), empty(N, torch.float32)
     sq.sq_smooth_quant_weight(W_t, None, sq.SQ_PER_CHANNEL, Wq, e)
     Y, mask, cnt = empty((M, N), torch.bfloat16), empty(K // 32, torch.int32), empty(1, torch.int32)
-    sq.llmint8_decomposed_linear_ex(X_t, W_t, Wq, e, thr, None, Y, mask, cnt, None,
+    acc = empty((M, N), torch.int32)
+    sq.llmint8_decomposed_linear_ex(X_t, W_t, Wq, e, thr, None, Y, mask, cnt, acc,
                                     sq.workspace(sq.SQ_OP_LLMINT8, M, N, K))
     sq.sq_sync_status()
     o = oracle.llmint8_linear(X, W, None, float(host(thr)[0]))
     assert o["count"] == 10 and int(host(cnt)[0]) == 10
     assert np.array_equal(host(mask).view(np.uint32), o["mask"])
-    assert np.array_equal(host_bits(Y), o["y_bf16"])
+    # the int8 part bit for bit; the sum with the outlier product (fp32 on the tensor cores,
+    # in an order the pages leave open) within the output tolerance of the fp64 reference
+    assert np.array_equal(host(acc), o["acc"])
     assert_close_bf16(host_bits(Y), o["y_ref"], "llmint8 with mean + 3 std")
 
 

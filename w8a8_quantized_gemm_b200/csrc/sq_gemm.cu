@@ -1,7 +1,7 @@
 // INT8 x INT8 -> INT32 GEMM on the sm_100a tensor cores (tcgen05.mma kind::i8) with a
 // fused dequantization / bias / bf16 epilogue, and the LLM.int8() outlier product
-// (tcgen05.mma kind::f16 on bf16 operands) accumulated into a second TMEM accumulator of
-// the same output tile and added in the same epilogue.
+// (tcgen05.mma kind::f16 on bf16 operands) added by the tensor cores onto the dequantized
+// fp32 values of the same output tile, which the epilogue writes back into TMEM.
 //
 // "量化基础与INT8" INT8推理流程 (INT8 (M,K) x (K,N) -> INT32 accumulate, INT32 -> 16-bit output)
 //   and 量化流程示例 (Y = Y_int32 * X_scale * W_scale);
@@ -17,13 +17,18 @@
 //   warp 1     allocates TMEM; one lane issues tcgen05.mma (4 x K=32 bytes per stage) into
 //              a double-buffered accumulator and frees stages with tcgen05.commit;
 //   warps 2-9  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one output row per
-//              thread, two column halves), y = (float(acc) * d_m) * e_n (+ o) (+ bias) -> bf16,
+//              thread, two column halves), y = (float(acc) * d_m) * e_n (+ bias) -> bf16,
 //              TMA stores through shared-memory staging; overlaps the next tile's main loop
 //              through the second TMEM buffer.
 // For a few tokens (M <= 64) the operands swap roles: the weight supplies the 128-row MMA
 // operand (output channels on TMEM lanes) and the tokens the N dimension, so no MMA row
 // and no weight byte is spent on padding; the epilogue then applies the per-token scale
 // per column and the per-channel scale and bias per row, and stores transposed boxes.
+// LLM.int8 (outlier operands): per tile the epilogue turns the int32 accumulator into
+// (float(acc) * d_m) * e_n + bias_n in place (tcgen05.st), the MMA warp then adds the bf16
+// outlier k-blocks onto it (fp32 accumulation), and the epilogue stores the sum; the outlier
+// k-blocks of tile i are issued after the first kOutlierLag int8 k-blocks of tile i+1, so the
+// accumulator stays double-buffered and neither product waits for the other.
 // Large shapes run on CTA pairs (clusters of 2): each pair computes a 256 x 256 tile with
 // tcgen05.mma.cta_group::2 issued by the even CTA; each CTA stages its own 128 rows of A
 // and 128 rows of B, the loads of both CTAs complete on the even CTA's barriers, and each
@@ -52,24 +57,39 @@ constexpr int kEpiBufs = 2;                   // per epilogue warp
 constexpr int kEpiSmem = kEpiWarps * kEpiBufs * kStageTileBytes;
 
 // PAIR: a CTA pair computes one 256 x BN tile; each CTA stages its 128 rows of A and half
-// of the BN rows of B, so a stage holds 32 KB instead of 48 and the ring gets 6 stages.
+// of the BN rows of B, so a stage holds 32 KB instead of 48 at BN = 256 and the ring gets
+// 6 stages.
+// TMEM: ACC_BUFS = 2 accumulators of BN columns each (columns [b*BN, (b+1)*BN)), so the
+// epilogue of tile i overlaps the main loop of tile i+1. With OUTLIERS (LLM.int8) the same
+// buffer serves both products of a tile: the int8 MMAs accumulate int32 there; the epilogue
+// converts it to the dequantized fp32 value (float(acc) * d_m) * e_n + bias_n and writes that
+// back into the same columns; the bf16 MMAs of the outlier columns then add their product onto
+// it (fp32 accumulation on the tensor cores), and the epilogue reads the sum and stores it as
+// bf16. The outlier MMAs of tile i are issued after the first kOutlierLag int8 k-blocks of
+// tile i+1, by which time the epilogue has written tile i back, so neither product waits for
+// the other in the common case.
+constexpr int pow2_cols(int c) { return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512; }
+constexpr int kOutlierLag = 8;
 template <int BN, bool OUTLIERS, int ACC_BUFS, bool PAIR = false>
 struct Cfg {
+  static constexpr int kBN = BN;
   static constexpr int kStageA = kBM * kBK;
   static constexpr int kStageB = (PAIR ? BN / 2 : BN) * kBK;
   static constexpr int kStageBytes = kStageA + kStageB;
   static constexpr int kStages = (192 * 1024) / kStageBytes;
-  static constexpr int kAccCols = OUTLIERS ? 2 * BN : BN;  // per buffer: int32 acc (+ fp32 acc)
-  static constexpr int kTmemCols = ACC_BUFS * kAccCols;
-  // with outlier operands but no outlier column at run time the int32 accumulator alone is
-  // needed, and the fp32 columns hold a second int32 buffer
-  static constexpr int kMaxBufs = (OUTLIERS && ACC_BUFS == 1) ? 2 : ACC_BUFS;
+  static constexpr int kUsedCols = ACC_BUFS * BN;
+  static constexpr int kTmemCols = pow2_cols(kUsedCols);  // allocations are powers of two
+  static constexpr int kChunksTotal = BN / 32;             // 32-column chunks of a tile
+  static constexpr int kChunks = (kChunksTotal + 1) / 2;   // per epilogue column half (at most)
   static constexpr int kBarOffset = kStages * kStageBytes + kEpiSmem;
   static constexpr int kSmemBytes = kBarOffset + 256 /*barriers*/ + 1024 /*alignment slack*/;
-  static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
+  static_assert(ACC_BUFS == 2, "double-buffered int32 accumulator");
+  static_assert(kUsedCols <= 512, "TMEM columns");
   static_assert(kStages >= 3, "pipeline depth");
   static_assert(kSmemBytes <= 232448, "shared memory");
-  static_assert(BN % 64 == 0, "two epilogue column halves of whole 32-column chunks");
+  static_assert(kStageB % 1024 == 0, "B tile of whole 128-byte swizzle atoms");
+  static_assert(BN % 32 == 0, "epilogue chunks of 32 columns");
+  static_assert(2 * kStages + 4 * ACC_BUFS + 1 <= 30, "barrier area");
 };
 
 struct Params {
@@ -96,6 +116,10 @@ struct Params {
   int32_t* partials;   // [tail tiles * splits][kEpiWarps][BN/64 chunks][8][32 lanes] int4 (int32 x4)
   int32_t* counters;   // [tail tiles * kEpiWarps] arrival counters, zero between calls
   const int32_t* o_count;
+  // short (programmatic) launches: the weight tiles of the CTA's first work unit are
+  // prefetched into L2 before the wait on the previous kernel (the weight does not depend
+  // on it in a decode step; a prefetch is only a hint, so it is safe even when it does)
+  int prefetch_weight;
   unsigned int* status;
   uint64_t wait_limit_ns;
   int fault;
@@ -265,8 +289,7 @@ __device__ __forceinline__ void dequant32_cols(const Params& p, const uint32_t (
   }
 }
 
-__device__ __forceinline__ void bias_pack32_cols(const Params& p, float (&y)[32], bool has_bias, int64_t n0,
-                                                 uint32_t (&out)[16]) {
+__device__ __forceinline__ void add_bias32_cols(const Params& p, float (&y)[32], bool has_bias, int64_t n0) {
   if (has_bias) {
 #pragma unroll
     for (int j = 0; j < 32; j += 8) {
@@ -280,6 +303,11 @@ __device__ __forceinline__ void bias_pack32_cols(const Params& p, float (&y)[32]
       }
     }
   }
+}
+
+__device__ __forceinline__ void bias_pack32_cols(const Params& p, float (&y)[32], bool has_bias, int64_t n0,
+                                                 uint32_t (&out)[16]) {
+  add_bias32_cols(p, y, has_bias, n0);
 #pragma unroll
   for (int j = 0; j < 16; ++j) out[j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
 }
@@ -342,6 +370,121 @@ __device__ __forceinline__ void store_box(const uint32_t (&v)[16], uint8_t* stag
   ebuf ^= 1;
 }
 
+// The single-thread roles walk the ring of shared-memory stages in the same order.
+struct Ring {
+  int stage;
+  uint32_t phase;
+  uint32_t issued_mask;    // producer: stages that received at least one load
+  uint32_t issued_parity;  // producer: parity of the last load issued into each stage
+  bool withheld;           // producer: the test hook's withheld stage
+};
+
+struct LoadCtx {
+  const Params* p;
+  const Abort* ab;
+  volatile int* abort_flag;
+  uint64_t* full;
+  uint64_t* empty;
+  uint8_t* stage_base;
+  bool leader;
+};
+
+// TMA producer: `count` k-blocks, block i at column x0 + i * x_step of map_a (rows ya) and
+// map_b (rows yb), each into the next stage once the MMAs have freed it.
+template <class C, bool PAIR>
+__device__ __forceinline__ bool load_blocks(Ring& r, const LoadCtx& c, const CUtensorMap* map_a,
+                                            const CUtensorMap* map_b, int x0, int x_step, int count, int ya,
+                                            int yb) {
+  const Params& p = *c.p;
+  for (int i = 0; i < count; ++i) {
+    if (!wait_or_abort(c.empty + r.stage, r.phase ^ 1, p.wait_limit_ns, c.abort_flag)) {
+      if (!*c.abort_flag) c.ab->raise(p.status, kErrProducerWait);
+      return false;
+    }
+    if (p.fault == 1 && !r.withheld) {
+      r.withheld = true;  // test hook: this stage never gets its loads nor its arrival
+    } else {
+      uint8_t* sa = c.stage_base + r.stage * C::kStageBytes;
+      uint8_t* sb = sa + C::kStageA;
+      const int x = x0 + i * x_step;
+      if constexpr (PAIR) {
+        // both CTAs' halves complete on the even CTA's barrier, which expects them all
+        if (c.leader) mbar_arrive_expect_tx(c.full + r.stage, 2 * C::kStageBytes);
+        const uint32_t fb = mapa_shared(c.full + r.stage, 0);
+        tma_load_2d_pair(sa, map_a, fb, x, ya, kEvictNormal);
+        tma_load_2d_pair(sb, map_b, fb, x, yb, kEvictNormal);
+      } else {
+        mbar_arrive_expect_tx(c.full + r.stage, C::kStageBytes);
+        tma_load_2d(sa, map_a, c.full + r.stage, x, ya, kEvictNormal);
+        tma_load_2d(sb, map_b, c.full + r.stage, x, yb, kEvictNormal);
+      }
+      r.issued_mask |= 1u << r.stage;
+      r.issued_parity = (r.issued_parity & ~(1u << r.stage)) | (r.phase << r.stage);
+    }
+    if (++r.stage == C::kStages) {
+      r.stage = 0;
+      r.phase ^= 1;
+    }
+  }
+  return true;
+}
+
+struct MmaCtx {
+  const Params* p;
+  const Abort* ab;
+  volatile int* abort_flag;
+  uint64_t* full;
+  uint64_t* empty;
+  uint8_t* stage_base;
+  uint32_t empty_c0, empty_c1;  // a pair's stage barriers in each CTA (shared::cluster)
+};
+
+// MMA issuer: `count` stages into the accumulator at d, int8 x int8 -> int32 (the first
+// instruction starts the accumulation when `start`), or with BF16 the outlier columns,
+// bf16 x bf16 added onto the fp32 values d holds. Each stage is freed by a commit.
+template <class C, bool PAIR, bool BF16>
+__device__ __forceinline__ bool mma_blocks(Ring& r, const MmaCtx& c, uint32_t d, int count, bool start) {
+  constexpr int kTileM = PAIR ? 2 * kBM : kBM;
+  constexpr uint32_t kIdesc = BF16 ? idesc_bf16_f32(kTileM, C::kBN) : idesc_i8_s32(kTileM, C::kBN);
+  const Params& p = *c.p;
+  for (int i = 0; i < count; ++i) {
+    if (!wait_or_abort(c.full + r.stage, r.phase, p.wait_limit_ns, c.abort_flag)) {
+      if (!*c.abort_flag) c.ab->raise(p.status, kErrMmaWait);
+      return false;
+    }
+    tc_fence_after();
+    const uint32_t a_addr = smem_u32(c.stage_base + r.stage * C::kStageBytes);
+    const uint32_t b_addr = a_addr + C::kStageA;
+#pragma unroll
+    for (int k = 0; k < kBK / 32; ++k) {
+      const uint32_t acc = (BF16 || !start || i != 0 || k != 0) ? 1u : 0u;
+      const uint64_t da = smem_desc_k128(a_addr + 32 * k), db = smem_desc_k128(b_addr + 32 * k);
+      if constexpr (PAIR) {
+        if constexpr (BF16)
+          mma_f16_pair(d, da, db, kIdesc, acc);
+        else
+          mma_i8_pair(d, da, db, kIdesc, acc);
+      } else {
+        if constexpr (BF16)
+          mma_f16(d, da, db, kIdesc, acc);
+        else
+          mma_i8(d, da, db, kIdesc, acc);
+      }
+    }
+    if constexpr (PAIR) {
+      mma_commit_pair(c.empty_c0 + 8u * r.stage);
+      mma_commit_pair(c.empty_c1 + 8u * r.stage);
+    } else {
+      mma_commit(c.empty + r.stage);
+    }
+    if (++r.stage == C::kStages) {
+      r.stage = 0;
+      r.phase ^= 1;
+    }
+  }
+  return true;
+}
+
 template <int BN, bool OUTLIERS, int ACC_BUFS, bool SWAP, bool ASYM, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -359,8 +502,10 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint64_t* full = bars;
   uint64_t* empty = bars + C::kStages;
   uint64_t* tmem_full = bars + 2 * C::kStages;
-  uint64_t* tmem_empty = tmem_full + C::kMaxBufs;
-  uint64_t* teardown = tmem_empty + C::kMaxBufs;
+  uint64_t* tmem_empty = tmem_full + ACC_BUFS;
+  uint64_t* y_ready = tmem_empty + ACC_BUFS;    // outlier form: dequantized values written back
+  uint64_t* tmem_full2 = y_ready + ACC_BUFS;    // outlier form: outlier product added
+  uint64_t* teardown = tmem_full2 + ACC_BUFS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
@@ -378,9 +523,13 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
-    for (int b = 0; b < C::kMaxBufs; ++b) {
+    for (int b = 0; b < ACC_BUFS; ++b) {
       mbar_init(tmem_full + b, 1);
       mbar_init(tmem_empty + b, PAIR ? 2 * kEpiWarps : kEpiWarps);
+    }
+    for (int b = 0; b < ACC_BUFS; ++b) {
+      mbar_init(y_ready + b, PAIR ? 2 * kEpiWarps : kEpiWarps);
+      mbar_init(tmem_full2 + b, 1);
     }
     mbar_init(teardown, 1);
     *abort_flag = 0;
@@ -392,6 +541,13 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     if (OUTLIERS) {
       tma_prefetch_desc(&tmXo);
       tma_prefetch_desc(&tmWo);
+    }
+    if (p.prefetch_weight && u_first < p.num_units) {
+      // the weight is the 128-row operand A when the operands are swapped, else B
+      const Unit w = unit_of(p, u_first);
+      const int y = SWAP ? (w.tile_mn % p.num_m_tiles) * kTileM + static_cast<int>(rank) * kBM
+                         : (w.tile_mn / p.num_m_tiles) * BN + (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
+      for (int kb = w.kb0; kb < w.kb1; ++kb) tma_prefetch_l2_2d(SWAP ? &tmA : &tmB, kb * kBK, y);
     }
   }
   if (warp == 1) {
@@ -417,66 +573,48 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const int num_units = p.num_units;
   int kb_o = 0;
   if constexpr (OUTLIERS) kb_o = (__ldg(p.o_count) + 63) / 64;
-  // accumulator buffers: double-buffered int32 when no outlier product is needed
-  const int acc_bufs = kb_o == 0 ? C::kMaxBufs : ACC_BUFS;
-  const uint32_t acc_cols = kb_o == 0 ? static_cast<uint32_t>(BN) : static_cast<uint32_t>(C::kAccCols);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued_mask = 0;      // stages that received at least one load
-      uint32_t issued_parity = 0;    // parity of the last load issued into each stage
-      bool withheld = false;
-      for (int u = u_first; u < num_units && !*abort_flag; u += u_step) {
-        const Unit w = unit_of(p, u);
-        const int m0 = (w.tile_mn % p.num_m_tiles) * kTileM + static_cast<int>(rank) * kBM;
-        const int n0 = (w.tile_mn / p.num_m_tiles) * BN + (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
-        const int kb0 = w.kb0, kb_i8 = w.kb1;
-        const int kb_total = kb_i8 + kb_o;
-        for (int kb = kb0; kb < kb_total; ++kb) {
-          if (!wait_or_abort(empty + stage, phase ^ 1, p.wait_limit_ns, abort_flag)) {
-            if (!*abort_flag) ab.raise(p.status, kErrProducerWait);
-            break;
-          }
-          if (p.fault == 1 && !withheld) {
-            withheld = true;  // test hook: this stage never gets its loads nor its arrival
-          } else {
-            uint8_t* sa = stage_base + stage * C::kStageBytes;
-            uint8_t* sb = sa + C::kStageA;
-            // int8 k-blocks of Xq / Wq, then bf16 k-blocks of the gathered outlier columns
-            // (64 bf16 = 128 bytes per row: the same stage geometry)
-            const bool body = kb < kb_i8;
-            const CUtensorMap* map_a = body ? &tmA : &tmXo;
-            const CUtensorMap* map_b = body ? &tmB : &tmWo;
-            const int x = body ? kb * kBK : (kb - kb_i8) * (kBK / 2);
-            if constexpr (PAIR) {
-              // both CTAs' halves complete on the even CTA's barrier, which expects them all
-              if (leader) mbar_arrive_expect_tx(full + stage, 2 * C::kStageBytes);
-              const uint32_t fb = mapa_shared(full + stage, 0);
-              tma_load_2d_pair(sa, map_a, fb, x, m0, kEvictNormal);
-              tma_load_2d_pair(sb, map_b, fb, x, n0, kEvictNormal);
-            } else {
-              mbar_arrive_expect_tx(full + stage, C::kStageBytes);
-              tma_load_2d(sa, map_a, full + stage, x, m0, kEvictNormal);
-              tma_load_2d(sb, map_b, full + stage, x, n0, kEvictNormal);
-            }
-            issued_mask |= 1u << stage;
-            issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-          }
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
+      Ring ring{};
+      const LoadCtx lc{&p, &ab, abort_flag, full, empty, stage_base, leader};
+      if (!OUTLIERS || kb_o == 0) {
+        // plain form: each unit's k-blocks in order
+        for (int u = u_first; u < num_units && !*abort_flag; u += u_step) {
+          const Unit w = unit_of(p, u);
+          const int m0 = (w.tile_mn % p.num_m_tiles) * kTileM + static_cast<int>(rank) * kBM;
+          const int n0 = (w.tile_mn / p.num_m_tiles) * BN + (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
+          if (!load_blocks<C, PAIR>(ring, lc, &tmA, &tmB, w.kb0 * kBK, kBK, w.kb1 - w.kb0, m0, n0)) break;
         }
+      } else {
+        // outlier form: the previous unit's outlier k-blocks (bf16, 64 columns = 128 bytes
+        // per row: the same stage geometry) after the first kOutlierLag int8 k-blocks of
+        // each unit, and the last unit's after the last unit
+        bool ok = true;
+        int j = 0, prev_m0 = 0, prev_n0 = 0;
+        for (int u = u_first; u < num_units && !*abort_flag; u += u_step, ++j) {
+          const Unit w = unit_of(p, u);
+          const int m0 = (w.tile_mn % p.num_m_tiles) * kTileM + static_cast<int>(rank) * kBM;
+          const int n0 = (w.tile_mn / p.num_m_tiles) * BN + (PAIR ? static_cast<int>(rank) * (BN / 2) : 0);
+          const int nk = w.kb1 - w.kb0;
+          const int ins = min(kOutlierLag, nk);
+          ok = load_blocks<C, PAIR>(ring, lc, &tmA, &tmB, w.kb0 * kBK, kBK, ins, m0, n0);
+          if (ok && j > 0) ok = load_blocks<C, PAIR>(ring, lc, &tmXo, &tmWo, 0, kBK / 2, kb_o, prev_m0, prev_n0);
+          if (ok) ok = load_blocks<C, PAIR>(ring, lc, &tmA, &tmB, (w.kb0 + ins) * kBK, kBK, nk - ins, m0, n0);
+          if (!ok) break;
+          prev_m0 = m0;
+          prev_n0 = n0;
+        }
+        if (ok && j > 0 && !*abort_flag)
+          load_blocks<C, PAIR>(ring, lc, &tmXo, &tmWo, 0, kBK / 2, kb_o, prev_m0, prev_n0);
       }
       // drain: every load this thread issued must have landed before the CTA exits (a
       // pair's odd CTA counts its copies on the even CTA's barriers, which the even CTA
       // drains before the final cluster barrier)
       for (int s = 0; s < C::kStages; ++s) {
-        if (leader && ((issued_mask >> s) & 1u)) {
-          if (!mbar_wait_bounded(full + s, (issued_parity >> s) & 1u, p.wait_limit_ns))
+        if (leader && ((ring.issued_mask >> s) & 1u)) {
+          if (!mbar_wait_bounded(full + s, (ring.issued_parity >> s) & 1u, p.wait_limit_ns))
             ab.raise(p.status, kErrTeardownWait);
         }
       }
@@ -484,76 +622,68 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && leader) {
-      constexpr uint32_t kIdescI8 = idesc_i8_s32(kTileM, BN);
-      constexpr uint32_t kIdescBf16 = idesc_bf16_f32(kTileM, BN);
       // a pair's commits go to the barrier in each CTA (shared::cluster addresses)
-      const uint32_t empty_c0 = PAIR ? mapa_shared(empty, 0) : 0u, empty_c1 = PAIR ? mapa_shared(empty, 1) : 0u;
       const uint32_t tfull_c0 = PAIR ? mapa_shared(tmem_full, 0) : 0u;
       const uint32_t tfull_c1 = PAIR ? mapa_shared(tmem_full, 1) : 0u;
-      int stage = 0;
-      uint32_t phase = 0;
+      const uint32_t tfull2_c0 = PAIR ? mapa_shared(tmem_full2, 0) : 0u;
+      const uint32_t tfull2_c1 = PAIR ? mapa_shared(tmem_full2, 1) : 0u;
+      Ring ring{};
+      const MmaCtx mc{&p, &ab, abort_flag, full, empty, stage_base, PAIR ? mapa_shared(empty, 0) : 0u,
+                      PAIR ? mapa_shared(empty, 1) : 0u};
+      auto commit_to = [&](uint64_t* bar, uint32_t c0, uint32_t c1, int b) {
+        if constexpr (PAIR) {
+          mma_commit_pair(c0 + 8u * b);
+          mma_commit_pair(c1 + 8u * b);
+        } else {
+          mma_commit(bar + b);
+        }
+      };
+      bool ok = true;
       int it = 0;
       for (int u = u_first; u < num_units && !*abort_flag; u += u_step, ++it) {
-        const int buf = it % acc_bufs;
-        const uint32_t acc_phase = (it / acc_bufs) & 1;
+        const int buf = it % ACC_BUFS;
+        const uint32_t acc_phase = (it / ACC_BUFS) & 1;
         if (!wait_or_abort(tmem_empty + buf, acc_phase ^ 1, p.wait_limit_ns, abort_flag)) {
           if (!*abort_flag) ab.raise(p.status, kErrMmaWait);
+          ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_i32 = tmem_base + buf * acc_cols;
-        const uint32_t d_f32 = d_i32 + BN;
+        const uint32_t d_i32 = tmem_base + buf * BN;
         const Unit w = unit_of(p, u);
-        const int kb0 = w.kb0, kb_i8 = w.kb1;
-        const int kb_total = kb_i8 + kb_o;
-        bool ok = true;
-        for (int kb = kb0; kb < kb_total; ++kb) {
-          if (!wait_or_abort(full + stage, phase, p.wait_limit_ns, abort_flag)) {
-            if (!*abort_flag) ab.raise(p.status, kErrMmaWait);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(stage_base + stage * C::kStageBytes);
-          const uint32_t b_addr = a_addr + C::kStageA;
-          if (kb < kb_i8) {
-#pragma unroll
-            for (int k = 0; k < kBK / 32; ++k) {
-              const uint32_t acc = (kb != kb0 || k != 0) ? 1u : 0u;
-              if constexpr (PAIR)
-                mma_i8_pair(d_i32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescI8, acc);
-              else
-                mma_i8(d_i32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescI8, acc);
+        const int nk = w.kb1 - w.kb0;
+        if (!OUTLIERS || kb_o == 0) {
+          ok = mma_blocks<C, PAIR, false>(ring, mc, d_i32, nk, true);
+        } else {
+          const int ins = min(kOutlierLag, nk);
+          ok = mma_blocks<C, PAIR, false>(ring, mc, d_i32, ins, true);
+          if (ok && it > 0) {
+            // the previous unit's outlier product starts once the epilogue has written its
+            // dequantized fp32 values back into its buffer
+            const int pit = it - 1;
+            ok = wait_or_abort(y_ready + pit % ACC_BUFS, (pit / ACC_BUFS) & 1, p.wait_limit_ns, abort_flag);
+            if (!ok && !*abort_flag) ab.raise(p.status, kErrMmaWait);
+            if (ok) {
+              tc_fence_after();
+              ok = mma_blocks<C, PAIR, true>(ring, mc, tmem_base + (pit % ACC_BUFS) * BN, kb_o, false);
             }
-          } else {
-            const int ko = kb - kb_i8;
-#pragma unroll
-            for (int k = 0; k < kBK / 32; ++k) {
-              const uint32_t acc = (ko | k) != 0 ? 1u : 0u;
-              if constexpr (PAIR)
-                mma_f16_pair(d_f32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescBf16, acc);
-              else
-                mma_f16(d_f32, smem_desc_k128(a_addr + 32 * k), smem_desc_k128(b_addr + 32 * k), kIdescBf16, acc);
-            }
+            if (ok) commit_to(tmem_full2, tfull2_c0, tfull2_c1, pit % ACC_BUFS);
           }
-          if constexpr (PAIR) {
-            mma_commit_pair(empty_c0 + 8u * stage);
-            mma_commit_pair(empty_c1 + 8u * stage);
-          } else {
-            mma_commit(empty + stage);
-          }
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
+          if (ok) ok = mma_blocks<C, PAIR, false>(ring, mc, d_i32, nk - ins, false);
         }
         if (!ok) break;
-        if constexpr (PAIR) {
-          mma_commit_pair(tfull_c0 + 8u * buf);
-          mma_commit_pair(tfull_c1 + 8u * buf);
-        } else {
-          mma_commit(tmem_full + buf);
+        commit_to(tmem_full, tfull_c0, tfull_c1, buf);
+      }
+      // the last unit's outlier product
+      if (OUTLIERS && kb_o > 0 && ok && it > 0 && !*abort_flag) {
+        const int pit = it - 1;
+        ok = wait_or_abort(y_ready + pit % ACC_BUFS, (pit / ACC_BUFS) & 1, p.wait_limit_ns, abort_flag);
+        if (!ok && !*abort_flag) ab.raise(p.status, kErrMmaWait);
+        if (ok) {
+          tc_fence_after();
+          ok = mma_blocks<C, PAIR, true>(ring, mc, tmem_base + (pit % ACC_BUFS) * BN, kb_o, false);
         }
+        if (ok) commit_to(tmem_full2, tfull2_c0, tfull2_c1, pit % ACC_BUFS);
       }
       // all MMAs issued by this thread complete before TMEM is released (in both CTAs of a
       // pair: the odd CTA frees its TMEM only after the final cluster barrier)
@@ -566,23 +696,26 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   } else {
     // ------------------------------------------------------------ epilogue
     // 8 warps: warp w reads TMEM lanes [32*(w%4), +32) (one output row per thread) and
-    // the column half (w-2)/4 of the tile, 32 columns at a time. The whole half-row is
-    // dequantized into registers (packed bf16) first, so the accumulator is handed back
-    // to the MMA warp before the stores; each 32x32 bf16 box then goes through this warp's
-    // staging buffer in shared memory to a TMA store.
-    constexpr int kChunks = BN / 64;  // 32-column chunks per warp
+    // the column half (w-2)/4 of the tile, 32 columns at a time (half 0 takes the first
+    // kChunks chunks, half 1 the rest: 4 + 4 at BN = 256, 3 + 2 at BN = 160). The whole
+    // half-row is dequantized into registers (packed bf16) first, so the accumulators are
+    // handed back to the MMA warp before the stores; each 32x32 bf16 box then goes through
+    // this warp's staging buffer in shared memory to a TMA store.
+    constexpr int kChunks = C::kChunks;  // 32-column chunks per warp (at most)
     static_assert(!(SWAP && OUTLIERS) && !(ASYM && OUTLIERS), "no outlier product with these forms");
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
+    const int my_chunks = half == 0 ? kChunks : C::kChunksTotal - kChunks;
     const int row = quad * 32 + lane;
     uint8_t* stage_tiles = epi_base + (warp - 2) * kEpiBufs * kStageTileBytes;
     int ebuf = 0;
     int it = 0;
-    // a pair's odd CTA hands the accumulator back on the even CTA's barrier
+    // a pair's odd CTA hands the accumulators back on the even CTA's barriers
     const uint32_t tempty_c0 = PAIR ? mapa_shared(tmem_empty, 0) : 0u;
+    const uint32_t yready_c0 = PAIR ? mapa_shared(y_ready, 0) : 0u;
     for (int u = u_first; u < num_units; u += u_step, ++it) {
-      const int buf = it % acc_bufs;
-      const uint32_t acc_phase = (it / acc_bufs) & 1;
+      const int buf = it % ACC_BUFS;
+      const uint32_t acc_phase = (it / ACC_BUFS) & 1;
       // everything that does not need the accumulator is fetched before waiting for it
       const Unit w = unit_of(p, u);
       const int tile_mn = w.tile_mn;
@@ -591,7 +724,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const int64_t r = m_tile0 + row;  // this thread's tile row (output row, or channel if swapped)
       const int64_t box_row0 = m_tile0 + quad * 32;
       const bool rows_live = box_row0 < p.rows;  // uniform across the warp
-      const int64_t n_half0 = static_cast<int64_t>(tile_mn / p.num_m_tiles) * BN + half * (BN / 2);
+      const int64_t n_half0 = static_cast<int64_t>(tile_mn / p.num_m_tiles) * BN + half * (kChunks * 32);
       const bool r_ok = r < p.rows;
       float row_scale = 0.0f, row_bias = 0.0f;
       int row_int = 0;
@@ -610,7 +743,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       // swapped operands spread the per-token column constants over the lanes; otherwise
       // the column constants are broadcast loads inside the chunk loop
       TokenConsts tc{};
-      if constexpr (SWAP) tc = load_token_consts<ASYM>(p, n_half0, lane, kChunks);
+      if constexpr (SWAP) tc = load_token_consts<ASYM>(p, n_half0, lane, my_chunks);
       const bool has_bias = p.bias != nullptr;
       // lane 0 waits and the warp follows its verdict, so the warp stays converged
       int ok = 0;
@@ -621,14 +754,94 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t t_row =
-          tmem_base + buf * acc_cols + (static_cast<uint32_t>(quad * 32) << 16) + half * (BN / 2);
-      if (!w.is_split) {
+      const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+      const uint32_t t_row = tmem_base + buf * BN + lane_off + half * (kChunks * 32);
+      if constexpr (OUTLIERS) {
+        // LLM.int8 form (tiles are never split). With outlier columns, pass 1 turns the int8
+        // product into its dequantized fp32 value (+ bias) in place and hands it to the MMA
+        // warp, whose bf16 MMAs add the outlier product onto it.
+        if (kb_o > 0) {
+#pragma unroll 1
+          for (int c = 0; c < my_chunks; ++c) {
+            const int64_t n0 = n_half0 + c * 32;
+            if (n0 >= p.cols) break;  // uniform across the warp
+            __syncwarp();
+            uint32_t acc[32];
+            tmem_ld_32x32b_x32(t_row + c * 32, acc);
+            tmem_wait_ld();
+            const int nvalid = (p.cols - n0) < 32 ? static_cast<int>(p.cols - n0) : 32;
+            if (p.acc_out != nullptr && r_ok) store_acc32<false>(p, acc, r, n0, nvalid);
+            float y[32];
+            dequant32_cols<false>(p, acc, row_scale, 0, n0, y);
+            add_bias32_cols(p, y, has_bias, n0);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[j] = __float_as_uint(y[j]);
+            tmem_st_32x32b_x32(t_row + c * 32, acc);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (PAIR)
+              mbar_arrive_remote(yready_c0 + 8u * buf);
+            else
+              mbar_arrive(y_ready + buf);
+          }
+          int ok2 = 0;
+          if (lane == 0) {
+            ok2 = wait_or_abort(tmem_full2 + buf, acc_phase, p.wait_limit_ns, abort_flag) ? 1 : 0;
+            if (!ok2 && !*abort_flag) ab.raise(p.status, kErrEpilogueWait);
+          }
+          ok2 = __shfl_sync(0xffffffffu, ok2, 0);
+          if (!ok2) break;
+          tc_fence_after();
+        }
+        // last pass: the sum with the outlier product (or, with no outlier column, the int8
+        // product dequantized here) -> packed bf16 in registers; the buffer is handed back
+        // before the stores
         uint32_t packed[kChunks][16];
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
           const int64_t n0 = n_half0 + c * 32;
-          if (n0 < p.cols) {  // uniform across the warp
+          if (c < my_chunks && n0 < p.cols) {  // uniform across the warp
+            __syncwarp();
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(t_row + c * 32, v);
+            tmem_wait_ld();
+            if (kb_o > 0) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                packed[c][j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+            } else {
+              const int nvalid = (p.cols - n0) < 32 ? static_cast<int>(p.cols - n0) : 32;
+              if (p.acc_out != nullptr && r_ok) store_acc32<false>(p, v, r, n0, nvalid);
+              float y[32];
+              dequant32_cols<false>(p, v, row_scale, 0, n0, y);
+              bias_pack32_cols(p, y, has_bias, n0, packed[c]);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (PAIR)
+            mbar_arrive_remote(tempty_c0 + 8u * buf);
+          else
+            mbar_arrive(tmem_empty + buf);
+        }
+        if (rows_live) {
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) {
+            const int64_t n0 = n_half0 + c * 32;
+            if (c < my_chunks && n0 < p.cols) store_box<false>(packed[c], stage_tiles, ebuf, lane, &tmY, n0, box_row0);
+          }
+        }
+      } else if (!w.is_split) {
+        uint32_t packed[kChunks][16];
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          const int64_t n0 = n_half0 + c * 32;
+          if (c < my_chunks && n0 < p.cols) {  // uniform across the warp
             __syncwarp();
             uint32_t acc[32];
             tmem_ld_32x32b_x32(t_row + c * 32, acc);
@@ -640,15 +853,6 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             else
               dequant32_cols<ASYM>(p, acc, row_scale, row_int, n0, y);
             if (p.acc_out != nullptr && r_ok) store_acc32<SWAP>(p, acc, r, n0, nvalid);
-            if constexpr (OUTLIERS) {
-              if (kb_o > 0) {
-                uint32_t of[32];  // fp32 outlier product of the same 32 columns
-                tmem_ld_32x32b_x32(t_row + BN + c * 32, of);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) y[j] = __fadd_rn(y[j], __uint_as_float(of[j]));
-              }
-            }
             if constexpr (SWAP)
               bias_pack32_tokens(y, has_bias, row_bias, packed[c]);
             else
@@ -668,7 +872,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
           for (int c = 0; c < kChunks; ++c) {
             const int64_t n0 = n_half0 + c * 32;
-            if (n0 < p.cols) store_box<SWAP>(packed[c], stage_tiles, ebuf, lane, &tmY, n0, box_row0);
+            if (c < my_chunks && n0 < p.cols) store_box<SWAP>(packed[c], stage_tiles, ebuf, lane, &tmY, n0, box_row0);
           }
         }
       } else {
@@ -684,7 +888,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
           const int64_t n0 = n_half0 + c * 32;
-          if (n0 < p.cols) {
+          if (c < my_chunks && n0 < p.cols) {
             __syncwarp();
             uint32_t acc[32];
             tmem_ld_32x32b_x32(t_row + c * 32, acc);
@@ -712,7 +916,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         if (last && rows_live) {
           __threadfence();
 #pragma unroll 1
-          for (int c = 0; c < kChunks; ++c) {
+          for (int c = 0; c < my_chunks; ++c) {
             const int64_t n0 = n_half0 + c * 32;
             if (n0 >= p.cols) break;
             const int nvalid = (p.cols - n0) < 32 ? static_cast<int>(p.cols - n0) : 32;
@@ -839,15 +1043,16 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool outliers) {
   const int64_t m_t = (rows + kBM - 1) / kBM;
   const int64_t kb = (K + kBK - 1) / kBK;
   auto tiles = [&](int bn) { return m_t * ((cols + bn - 1) / bn); };
+  constexpr int wide = 256;
   Plan pl{swap, false, 64, 0, 0, 1, static_cast<int>(kb)};
   if (swap) {
     pl.bn = 64;
-  } else if (tiles(256) >= kPlanSms) {
-    pl.bn = 256;
-    // CTA pairs when the 256 x 256 tiles still give every pair of SMs a tile and add no
+  } else if (tiles(wide) >= kPlanSms) {
+    pl.bn = wide;
+    // CTA pairs when the 256-row tiles still give every pair of SMs a tile and add no
     // padded rows (an even number of 128-row tiles) or few (at least 32 of them): with
     // 65..128 rows, say, the odd CTA of every pair would only compute padding
-    const int64_t pair_tiles = ((rows + 2 * kBM - 1) / (2 * kBM)) * ((cols + 255) / 256);
+    const int64_t pair_tiles = ((rows + 2 * kBM - 1) / (2 * kBM)) * ((cols + wide - 1) / wide);
     const bool pair_rows = m_t % 2 == 0 || m_t >= 32;
     if (pair_rows && pair_tiles >= kPlanSms / 2) {
       pl.pair = true;
@@ -949,6 +1154,7 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   }
   p.o_count = a.o_count;
   p.status = device_status_word();
+  p.prefetch_weight = (SWAP || pl.tail_tiles > 0) ? 1 : 0;
   p.wait_limit_ns = a.wait_limit_ns;
   p.fault = a.fault;
   // one persistent CTA per SM (a pair per two SMs)
@@ -989,9 +1195,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream, const char** why
   if (gemv_applies(a.M, a.K, outliers) && a.fault == 0) return launch_gemv(a, stream);
   const Plan pl = plan_gemm(a.M, a.N, a.K, outliers);
   if (outliers) {
-    // int32 + fp32 accumulators: 256-wide tiles fit TMEM once, narrower ones twice
-    if (pl.pair) return run<256, true, 1, false, false, true>(a, pl, stream, why);
-    if (pl.bn == 256) return run<256, true, 1, false>(a, pl, stream, why);
+    if (pl.pair) return run<256, true, 2, false, false, true>(a, pl, stream, why);
+    if (pl.bn == 256) return run<256, true, 2, false>(a, pl, stream, why);
     if (pl.bn == 128) return run<128, true, 2, false>(a, pl, stream, why);
     return run<64, true, 2, false>(a, pl, stream, why);
   }

@@ -13,6 +13,7 @@
 // The epilogue is exactly the GEMM's: y = bf16_rne((float(acc) * d_m) * e_n + bias_n), the
 // accumulator first corrected by acc - z_m * rowsum_n for asymmetric activations.
 #include "sq_internal.h"
+#include "sq_ptx.cuh"
 
 #include <cuda_bf16.h>
 
@@ -38,6 +39,13 @@ gemv_i8_kernel(const int8_t* __restrict__ Xq, const int8_t* __restrict__ Wq, con
                uint16_t* __restrict__ Y, int32_t* __restrict__ acc_out, int M, int64_t N, int64_t K) {
   constexpr int kGemvUnroll = gemv_unroll<MT>();
   extern __shared__ int4 xs[];  // [MT][K/16], rows past M zero
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (kGemvThreads / 32);
+  const int64_t n_first = static_cast<int64_t>(blockIdx.x) * (kGemvThreads / 32) + (threadIdx.x >> 5);
+  // the weight does not depend on the previous kernel in a decode step: each warp starts
+  // bringing its first channel row into L2 before waiting for that kernel (a prefetch is a
+  // hint, safe even when the previous kernel wrote the weight)
+  if (lane == 0 && n_first < N) bulk_prefetch_l2(Wq + n_first * K, static_cast<uint32_t>(K));
   griddep_wait();
   griddep_launch_dependents();
   const int64_t vecs = K / 16;
@@ -46,9 +54,7 @@ gemv_i8_kernel(const int8_t* __restrict__ Xq, const int8_t* __restrict__ Wq, con
     xs[i] = m < M ? __ldg(reinterpret_cast<const int4*>(Xq + m * K) + (i - m * vecs)) : make_int4(0, 0, 0, 0);
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * (kGemvThreads / 32);
-  for (int64_t n = static_cast<int64_t>(blockIdx.x) * (kGemvThreads / 32) + (threadIdx.x >> 5); n < N; n += warps) {
+  for (int64_t n = n_first; n < N; n += warps) {
     const int4* wrow = reinterpret_cast<const int4*>(Wq + n * K);
     int acc[MT];
 #pragma unroll

@@ -21,7 +21,10 @@ ROW_SHAPES = [(1, 16), (3, 48), (5, 512), (4, 528), (9, 1024), (7, 2048), (6, 40
               (2, 16384), (2, 20000), (1, 65536)]
 
 
-@pytest.mark.parametrize("M,K", [(1, 16), (7, 48), (33, 272), (300, 4112), (2048, 4096), (129, 8192)])
+# column blocks of 64 / 128 / 256 columns (the kernel picks by K and SM count), clusters of
+# 1 to 8 CTAs along the rows (at least 64 rows each), ragged last blocks and row splits
+@pytest.mark.parametrize("M,K", [(1, 16), (7, 48), (33, 272), (300, 4112), (2048, 4096), (129, 8192), (600, 8192),
+                                 (520, 8208), (5000, 1024)])
 def test_channel_absmax_exact(M, K):
     p = wl.random_problem(M, 8, K, seed=M + K, outliers=3, offset=50.0)
     amax = empty(K, torch.float32)
@@ -44,7 +47,7 @@ def test_channel_absmax_strided():
 
 
 @pytest.mark.parametrize("alpha", [0.0, 0.3, 0.5, 0.7, 1.0])
-@pytest.mark.parametrize("N,K", [(24, 96), (300, 4096)])
+@pytest.mark.parametrize("N,K", [(24, 96), (300, 4096), (1000, 8192), (11008, 4096)])
 def test_smooth_scale_within_one_ulp(alpha, N, K):
     p = wl.random_problem(64, N, K, seed=N, outliers=4, offset=40.0)
     amax = oracle.act_channel_absmax(p.X)

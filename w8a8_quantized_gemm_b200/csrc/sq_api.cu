@@ -152,8 +152,8 @@ sq_status sq_smooth_scale(const float* act_amax, const void* W_bf16, int64_t N, 
   if (static_cast<const void*>(s) == static_cast<const void*>(act_amax) || s == inv_s)
     return fail(SQ_ERR_INVALID, "%s: s must not alias act_amax or inv_s", fn);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = sq::launch_col_absmax(static_cast<const uint16_t*>(W_bf16), N, K, ldw, s, false, cs);
-  if (e == cudaSuccess) e = sq::launch_smooth_factors(act_amax, s, inv_s, K, alpha, cs);
+  cudaError_t e =
+      sq::launch_smooth_scale(act_amax, static_cast<const uint16_t*>(W_bf16), N, K, ldw, alpha, s, inv_s, cs);
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
 }
 

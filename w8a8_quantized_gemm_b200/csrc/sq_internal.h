@@ -94,13 +94,13 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 // ---- reductions (sq_reduce.cu)
 // words[0..n) = 0.
 cudaError_t launch_zero_words(uint32_t* words, int64_t n, cudaStream_t stream);
-// Column absmax of a bf16 [rows, K] matrix into amax (fp32 [K], stored as ordered bits).
-// With accumulate == 0 the output is reset first.
+// Column absmax of a bf16 [rows, K] matrix into amax (fp32 [K]); with `accumulate` the
+// maximum with the values amax already holds. One launch, no reset.
 cudaError_t launch_col_absmax(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, float* amax,
                               bool accumulate, cudaStream_t stream);
-// s/inv_s from act_amax and the column absmax of W already stored in s (in place).
-cudaError_t launch_smooth_factors(const float* act_amax, float* s_inout, float* inv_s, int64_t K, float alpha,
-                                  cudaStream_t stream);
+// Smoothing factors s / inv_s from act_amax and the column absmax of W, in one pass over W.
+cudaError_t launch_smooth_scale(const float* act_amax, const uint16_t* W, int64_t N, int64_t K, int64_t ldw,
+                                float alpha, float* s, float* inv_s, cudaStream_t stream);
 
 // ---- row quantization (sq_quant.cu)
 struct OutlierView {

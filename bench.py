@@ -39,10 +39,13 @@ THRESHOLD = 6.0
 N_SETS = 4  # rotating input sets: 4 x (16.8 MB X + 90.2 MB W) = 428 MB > 126 MB L2
 
 # DRAM traffic of one int8 GEMM launch on this workload (dram__bytes_read.sum +
-# dram__bytes_write.sum of an ncu capture of `python -m w8a8_quantized_gemm_b200.profile_cases
-# gemm`), valid while the GEMM source's code (comments aside) hashes to GEMM_SRC_SHA.
-NCU_GEMM_TRAFFIC_BYTES = 53596928 + 13500928
-GEMM_SRC_SHA = "3f0e8e578675aa01"
+# dram__bytes_write.sum of `ncu --clock-control none --metrics gpu__time_duration.sum,
+# dram__bytes_read.sum,dram__bytes_write.sum -k regex:w8a8_gemm -s 1 -c 1 python -m
+# w8a8_quantized_gemm_b200.profile_cases gemm`), valid while the GEMM source's code (comments
+# aside) hashes to GEMM_SRC_SHA. The reads are Xq + Wq once (53.6 MB); most of Y's 45 MB of
+# writes are still in L2 when the kernel ends, so the write figure is below Y's size.
+NCU_GEMM_TRAFFIC_BYTES = 53633024 + 13139712
+GEMM_SRC_SHA = "cbe14453b03f694d"
 
 
 def _peaks():
@@ -346,6 +349,10 @@ def run_ours(args):
     per_kernel = path.collect(records)
     del graph
     iso = path.isolated_times()
+    try:
+        ktimes = measure_kernel_times(path)
+    except Exception as exc:  # the profiler's activity records are a diagnostic: keep the line
+        ktimes = {"error": f"{type(exc).__name__}: {exc}"}
 
     ms_step = ms_total / args.steps
     value = whole_job_rate(ops_step, args.steps, ws, ms_total) / 1e12
@@ -383,6 +390,16 @@ def run_ours(args):
             ent.update({"TOPS": round(tops, 1), "frac_int8_peak": round(tops / int8_peak, 4), "k_outliers": k_o})
         kernels[n] = ent
 
+    # the library's kernels inside the step (several per call), from the profiler's records;
+    # the masked LLM.int8 quantization is rated on the bytes it must move: X read, codes and
+    # row scales written, both gathered outlier operands (zero-padded to 64 columns) written
+    # and the outlier columns of W read
+    pad = (k_o + 63) // 64 * 64
+    masked_bytes = 3.0 * M * K + 4 * M + 2.0 * (M + N) * pad + 2.0 * N * k_o
+    ktimes_note = ("avg device time per launch over 4 untimed steps (CUDA profiler activity records); "
+                   f"the masked quantization of the LLM.int8 linear moves {masked_bytes / 1e6:.1f} MB "
+                   f"(X read, codes, row scales, both gathered outlier operands, the {k_o} outlier columns of W)")
+
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = run_e2e(path, p, args, ops_step, use_dist, local, ws)
 
@@ -395,7 +412,8 @@ def run_ours(args):
                    "M": M, "N": N, "K": K, "outlier_columns": k_o, "ops_per_step": ops_step,
                    "l2": f"{N_SETS} rotating input sets ({N_SETS * (2 * M * K + 2 * N * K) / 1e6:.0f} MB) > L2",
                    "parallelism": f"replica x{ws}"},
-        "roofline": roofline, "kernels": kernels, "gpu_launches": int(launches), "launch_mode": mode,
+        "roofline": roofline, "kernels": kernels, "kernel_times_in_step": ktimes,
+        "kernel_times_note": ktimes_note, "gpu_launches": int(launches), "launch_mode": mode,
         "kernel_timing": f"roofline: CUDA event nodes around each operation of every {args.sample_every}th timed "
                          f"step ({len(records)} steps sampled); kernels: us / rate / frac from each operation "
                          f"timed alone over the {N_SETS} input sets in its own CUDA graph, us_in_step from the "
@@ -409,6 +427,14 @@ def run_ours(args):
             line["other_workloads"] = measure_configs(dev, hbm, int8_peak)
         except Exception as exc:  # keep the main line; say what failed
             line["other_workloads"] = {"error": f"{type(exc).__name__}: {exc}"}
+        torch.cuda.empty_cache()
+        try:
+            pk = measure_int8_peak(dev, iso["int8_gemm_dequant"] * 1e3)
+            line["int8_peak_measured"] = pk
+            burst = pk["cublas_int8_8192^3"]["burst_TOPS"]
+            roofline["frac_of_cublas_int8_burst"] = round(gemm_tops / burst, 4)
+        except Exception as exc:
+            line["int8_peak_measured"] = {"error": f"{type(exc).__name__}: {exc}"}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(p, args.cpu_budget)
     if use_dist:
@@ -444,20 +470,7 @@ def _graph_time_us(torch, fns, reps):
     return a.elapsed_time(b) * 1e3 / (reps * len(fns))
 
 
-def measure_configs(dev, hbm, int8_peak):
-    """The other workloads, each timed alone after the main timed region (not part of the
-    step): the decode sweep (M in {1,4,16,64}, 4096 x 4096, eight weight copies rotated so the
-    weight streams from HBM), the LLM.int8 sweep (X [4096, 8192] with 0 / 8 / 82 outlier
-    columns, W [8192, 8192]), the 70B-shaped FFN GEMM (8192 x 28672 x 8192) and the variants
-    on X [8192, 8192] (two rotated copies, 268 MB > L2). Random device inputs of those shapes
-    and distributions; the parity tests cover the values."""
-    import torch
-
-    from w8a8_quantized_gemm_b200 import sq
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(0)
-    out = {}
-
+def _entries(hbm, int8_peak):
     def hbm_entry(us, nbytes):
         gbs = nbytes / (us * 1e-6) / 1e9
         return {"us": round(us, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
@@ -465,12 +478,76 @@ def measure_configs(dev, hbm, int8_peak):
     def tops_entry(us, ops):
         t = ops / (us * 1e-6) / 1e12
         return {"us": round(us, 2), "TOPS": round(t, 1), "frac_int8_peak": round(t / int8_peak, 4)}
+    return hbm_entry, tops_entry
 
-    # decode sweep: bytes N*K + M*K + 2*M*N + 4*(M+N) per call
+
+def measure_int8_peak(dev, gemm_us_7b):
+    """cuBLAS's int8 GEMM (torch._int_mm, int32 output) as a measured int8 tensor-core rate:
+    8192^3 best of ten graph replays (burst) and back to back for about two seconds
+    (sustained, under the power cap), and on the 2048 x 11008 x 4096 shape beside this
+    library's GEMM (which also dequantizes and writes bf16). A library kernel, timed here as a
+    reference rate only; it is not on the hot path."""
+    import torch
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1)
+    out = {}
+    n = 8192
+    A = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=gen)
+    B = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=gen)
+    C = torch.empty((n, n), dtype=torch.int32, device=dev)
+    Bt = B.t()
+    fn = [lambda: torch._int_mm(A, Bt, out=C)]
+    best = min(_graph_time_us(torch, fn, 3) for _ in range(10))
+    reps = max(3, int(2.0e6 / best))
+    sustained = _graph_time_us(torch, fn, reps)
+    ops = 2.0 * n ** 3
+    out["cublas_int8_8192^3"] = {"burst_us": round(best, 1), "burst_TOPS": round(ops / best / 1e6, 1),
+                                 "sustained_us": round(sustained, 1),
+                                 "sustained_TOPS": round(ops / sustained / 1e6, 1),
+                                 "sustained_reps": reps}
+    del A, B, C, Bt
+    M, N, K = 2048, 11008, 4096
+    Xq = [torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev, generator=gen) for _ in range(4)]
+    Wq = [torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev, generator=gen) for _ in range(4)]
+    C = torch.empty((M, N), dtype=torch.int32, device=dev)
+    us = _graph_time_us(torch, [(lambda x=x, w=w: torch._int_mm(x, w.t(), out=C)) for x, w in zip(Xq, Wq)], 10)
+    burst = ops / best / 1e6
+    out["cublas_int8_2048x11008x4096"] = {"us": round(us, 2), "TOPS": round(2.0 * M * N * K / us / 1e6, 1)}
+    out["w8a8_gemm_2048x11008x4096"] = {"us": round(gemm_us_7b, 2),
+                                        "TOPS": round(2.0 * M * N * K / gemm_us_7b / 1e6, 1),
+                                        "frac_of_cublas_int8_burst": round(2.0 * M * N * K / gemm_us_7b / 1e6 / burst,
+                                                                           4)}
+    out["note"] = ("cuBLAS writes int32 (4 bytes per output); the library's GEMM dequantizes and writes bf16 "
+                   "(2 bytes); both are timed in CUDA graphs over rotated inputs")
+    return out
+
+
+def measure_configs(dev, hbm, int8_peak):
+    """The other workloads, each timed alone after the main timed region (not part of the
+    step): the tiny config's latency, the decode sweep (M in {1,4,16,64}, 4096 x 4096, eight
+    weight copies rotated so the weight streams from HBM; the GEMM alone and the decode step
+    quantization + GEMM), the LLM.int8 sweep (X [4096, 8192] with 0 / 8 / 82 outlier columns,
+    W [8192, 8192]), the 70B-shaped FFN path (8192 x 28672 x 8192: calibration, smoothing,
+    both quantizations and the GEMM at alpha 0.3 / 0.5 / 0.7, and the GEMM forms) and the
+    reductions and variants on large inputs (X [8192, 8192], two rotated copies, 268 MB > L2).
+    Random device inputs of those shapes and distributions; the parity tests cover the values."""
+    import torch
+
+    from w8a8_quantized_gemm_b200 import sq
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    out = {}
+    hbm_entry, tops_entry = _entries(hbm, int8_peak)
+
+    out["tiny_latency"] = measure_tiny_latency(dev)
+
+    # decode sweep: bytes N*K + M*K + 2*M*N + 4*(M+N) per GEMM call; the step adds the
+    # activation rows (2*M*K read, M*K + 4*M written)
     N = K = 4096
     Wqs = [torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev, generator=gen) for _ in range(8)]
     e = torch.rand(N, device=dev, generator=gen) * 1e-3
-    dec = {}
+    inv_s = torch.rand(K, device=dev, generator=gen) + 0.5
+    dec, dec_path = {}, {}
     for M in (1, 4, 16, 64):
         Xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev, generator=gen)
         d = torch.rand(M, device=dev, generator=gen) * 1e-2
@@ -478,8 +555,23 @@ def measure_configs(dev, hbm, int8_peak):
         ws = sq.workspace(sq.SQ_OP_INT8_GEMM_DEQUANT, M, N, K, device=dev)
         us = _graph_time_us(torch, [(lambda w=w: sq.sq_int8_gemm_dequant(Xq, w, d, e, sq.SQ_PER_CHANNEL, None, Y,
                                                                          None, ws)) for w in Wqs], 10)
-        dec[f"M{M}"] = hbm_entry(us, N * K + M * K + 2 * M * N + 4 * (M + N))
+        gemm_bytes = N * K + M * K + 2 * M * N + 4 * (M + N)
+        dec[f"M{M}"] = hbm_entry(us, gemm_bytes)
+        Xs = [torch.randn(M, K, device=dev, generator=gen) for _ in range(8)]
+        for x in Xs:
+            x[:, :6] += 40.0
+        Xs = [x.to(torch.bfloat16) for x in Xs]
+        Xq2, d2 = torch.empty((M, K), dtype=torch.int8, device=dev), torch.empty(M, device=dev)
+
+        def step(x, w, Xq2=Xq2, d2=d2, Y=Y, ws=ws):
+            sq.sq_quant_act_per_token(x, inv_s, Xq2, d2)
+            sq.sq_int8_gemm_dequant(Xq2, w, d2, e, sq.SQ_PER_CHANNEL, None, Y, None, ws)
+        us2 = _graph_time_us(torch, [(lambda x=x, w=w: step(x, w)) for x, w in zip(Xs, Wqs)], 10)
+        ent = hbm_entry(us2, gemm_bytes + 3 * M * K + 4 * M)
+        ent["launches"] = 2
+        dec_path[f"M{M}"] = ent
     out["decode_4096x4096"] = dec
+    out["decode_step_quant_gemm_4096x4096"] = dec_path
     del Wqs
 
     # LLM.int8 sweep
@@ -508,31 +600,9 @@ def measure_configs(dev, hbm, int8_peak):
     out["llmint8_4096x8192x8192"] = llm
     del base, W, Wq, Y, ws, X
 
-    # 70B-shaped FFN GEMM with bias
-    M, N, K = 8192, 28672, 8192
-    Xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev, generator=gen)
-    Wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev, generator=gen)
-    d = torch.rand(M, device=dev, generator=gen) * 1e-2
-    e = torch.rand(N, device=dev, generator=gen) * 1e-3
-    bias = (0.1 * torch.randn(N, device=dev, generator=gen)).to(torch.bfloat16)
-    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    us = _graph_time_us(torch, [lambda: sq.sq_int8_gemm_dequant(Xq, Wq, d, e, sq.SQ_PER_CHANNEL, bias, Y)], 3)
-    out["ffn70b_gemm_8192x28672x8192"] = tops_entry(us, 2.0 * M * N * K)
-    # the GEMM with asymmetric activations and with a per-tensor activation scale, same shape
-    z = torch.randint(-128, 128, (M,), dtype=torch.int32, device=dev, generator=gen)
-    rs = torch.empty(N, dtype=torch.int32, device=dev)
-    sq.sq_weight_row_sums(Wq, rs)
-    us = _graph_time_us(torch, [lambda: sq.sq_int8_gemm_dequant_ex(Xq, Wq, d, sq.SQ_PER_CHANNEL, z, e,
-                                                                   sq.SQ_PER_CHANNEL, rs, bias, Y)], 3)
-    out["gemm_asymmetric_8192x28672x8192"] = tops_entry(us, 2.0 * M * N * K)
-    us = _graph_time_us(torch, [lambda: sq.sq_int8_gemm_dequant_ex(Xq, Wq, d[:1], sq.SQ_PER_TENSOR, None, e,
-                                                                   sq.SQ_PER_CHANNEL, None, bias, Y)], 3)
-    out["gemm_per_tensor_x_8192x28672x8192"] = tops_entry(us, 2.0 * M * N * K)
-    us = _graph_time_us(torch, [lambda: sq.sq_weight_row_sums(Wq, rs)], 5)
-    out["weight_row_sums_28672x8192"] = hbm_entry(us, N * K + 4 * N)
-    del Xq, Wq, Y
+    out.update(measure_ffn70b(dev, hbm, int8_peak, gen))
 
-    # variants on X [8192, 8192]: algorithmic bytes read X once (+ write codes once)
+    # reductions and variants on X [8192, 8192]: algorithmic bytes read X once (+ write codes once)
     M = K = 8192
     Xs = [(1.5 * torch.randn(M, K, device=dev, generator=gen) + 0.2).to(torch.bfloat16) for _ in range(2)]
     inv = torch.rand(K, device=dev, generator=gen) + 0.5
@@ -541,12 +611,14 @@ def measure_configs(dev, hbm, int8_peak):
     Xq = torch.empty((M, K), dtype=torch.int8, device=dev)
     d, z = torch.empty(M, device=dev), torch.empty(M, dtype=torch.int32, device=dev)
     d1, clip, thr = torch.empty(1, device=dev), torch.full((1,), 4.0, device=dev), torch.empty(1, device=dev)
+    amax = torch.empty(K, device=dev)
     wpt = sq.workspace(sq.SQ_OP_QUANT_ACT_PER_TENSOR, M, 0, K, device=dev)
     wms = sq.workspace(sq.SQ_OP_MEAN_STD_THRESHOLD, M, 0, K, device=dev)
     wpc = sq.workspace(sq.SQ_OP_ABS_PERCENTILE, M, 0, K, device=dev)
     n = M * K
     var = {}
     cases = [
+        ("act_channel_absmax", 2 * n + 4 * K, lambda X: sq.sq_act_channel_absmax(X, amax)),
         ("quant_act_per_token", 3 * n, lambda X: sq.sq_quant_act_per_token(X, inv, Xq, d)),
         ("layernorm_smooth_quant", 3 * n, lambda X: sq.sq_norm_smooth_quant(X, sq.SQ_NORM_LAYER, g, b, 1e-5, inv, Xq,
                                                                             d)),
@@ -565,6 +637,150 @@ def measure_configs(dev, hbm, int8_peak):
                    "dynamic per-tensor form reads X twice by design (global maximum first)")
     out["variants_8192x8192"] = var
     sq.sq_sync_status()
+    return out
+
+
+def measure_ffn70b(dev, hbm, int8_peak, gen):
+    """The 70B-shaped FFN path, X [8192, 8192] ~N(0,1) with 4 columns x100, W [28672, 8192]
+    ~N(0,0.01), bias ~N(0,0.1): for alpha in {0.3, 0.5, 0.7} each call of the SmoothQuant path
+    (channel absmax of X, smoothing factors from W, smoothed per-channel weight quantization,
+    smoothed per-token activation quantization, GEMM + dequant + bias) timed alone, and the
+    whole path as one graph; then the GEMM with asymmetric activations, with a per-tensor
+    activation scale, and the weight row sums."""
+    import torch
+
+    from w8a8_quantized_gemm_b200 import sq
+    hbm_entry, tops_entry = _entries(hbm, int8_peak)
+    out = {}
+    M, N, K = 8192, 28672, 8192
+    X = torch.randn(M, K, device=dev, generator=gen)
+    cols = torch.randperm(K, device=dev, generator=gen)[:4]
+    X[:, cols] *= 100.0
+    X = X.to(torch.bfloat16)
+    W = (0.01 * torch.randn(N, K, device=dev, generator=gen)).to(torch.bfloat16)
+    bias = (0.1 * torch.randn(N, device=dev, generator=gen)).to(torch.bfloat16)
+    amax, s, inv_s = (torch.empty(K, device=dev) for _ in range(3))
+    Wq, e = torch.empty((N, K), dtype=torch.int8, device=dev), torch.empty(N, device=dev)
+    Xq, d = torch.empty((M, K), dtype=torch.int8, device=dev), torch.empty(M, device=dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ops = 2.0 * M * N * K
+    path = {}
+    for alpha in (0.3, 0.5, 0.7):
+        steps = {
+            "act_channel_absmax": (lambda: sq.sq_act_channel_absmax(X, amax), hbm, 2 * M * K + 4 * K),
+            "smooth_scale": (lambda: sq.sq_smooth_scale(amax, W, alpha, s, inv_s), hbm, 2 * N * K + 12 * K),
+            "smooth_quant_weight": (lambda: sq.sq_smooth_quant_weight(W, s, sq.SQ_PER_CHANNEL, Wq, e), hbm,
+                                    3 * N * K + 4 * N + 4 * K),
+            "quant_act_per_token": (lambda: sq.sq_quant_act_per_token(X, inv_s, Xq, d), hbm, 3 * M * K + 4 * M + 4 * K),
+            "int8_gemm_dequant_bias": (lambda: sq.sq_int8_gemm_dequant(Xq, Wq, d, e, sq.SQ_PER_CHANNEL, bias, Y),
+                                       None, ops),
+        }
+        ent = {}
+        total = 0.0
+        for name, (fn, bw, work) in steps.items():
+            us = _graph_time_us(torch, [fn], 3)
+            total += us
+            ent[name] = hbm_entry(us, work) if bw is not None else tops_entry(us, work)
+
+        def whole():
+            for fn, _, _ in steps.values():
+                fn()
+        us = _graph_time_us(torch, [whole], 3)
+        ent["whole_path"] = tops_entry(us, ops)
+        ent["whole_path"]["sum_of_calls_us"] = round(total, 1)
+        path[f"alpha={alpha}"] = ent
+    out["ffn70b_path_8192x28672x8192"] = path
+    us = _graph_time_us(torch, [lambda: sq.sq_int8_gemm_dequant(Xq, Wq, d, e, sq.SQ_PER_CHANNEL, bias, Y)], 3)
+    out["ffn70b_gemm_8192x28672x8192"] = tops_entry(us, ops)
+    z = torch.randint(-128, 128, (M,), dtype=torch.int32, device=dev, generator=gen)
+    rs = torch.empty(N, dtype=torch.int32, device=dev)
+    sq.sq_weight_row_sums(Wq, rs)
+    us = _graph_time_us(torch, [lambda: sq.sq_int8_gemm_dequant_ex(Xq, Wq, d, sq.SQ_PER_CHANNEL, z, e,
+                                                                   sq.SQ_PER_CHANNEL, rs, bias, Y)], 3)
+    out["gemm_asymmetric_8192x28672x8192"] = tops_entry(us, ops)
+    us = _graph_time_us(torch, [lambda: sq.sq_int8_gemm_dequant_ex(Xq, Wq, d[:1], sq.SQ_PER_TENSOR, None, e,
+                                                                   sq.SQ_PER_CHANNEL, None, bias, Y)], 3)
+    out["gemm_per_tensor_x_8192x28672x8192"] = tops_entry(us, ops)
+    us = _graph_time_us(torch, [lambda: sq.sq_weight_row_sums(Wq, rs)], 5)
+    out["weight_row_sums_28672x8192"] = hbm_entry(us, N * K + 4 * N)
+    return out
+
+
+def measure_tiny_latency(dev):
+    """The tiny config's whole SmoothQuant path (channel absmax, smoothing factors, per-tensor
+    weight quantization, per-token activation quantization, GEMM) and its LLM.int8 linear,
+    X [16, 256], W [256, 256]: launch-to-result latency of one eager call sequence (host clock
+    from the first launch to the end of a stream synchronize, median of 50) and the device
+    time of the same sequence replayed as a CUDA graph."""
+    import torch
+
+    from w8a8_quantized_gemm_b200 import sq
+    p = wl.tiny()
+    M, N, K = p.M, p.N, p.K
+
+    def up(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    X, W = up(p.X), up(p.W)
+    amax, s, inv_s = (torch.empty(K, device=dev) for _ in range(3))
+    Wq, e = torch.empty((N, K), dtype=torch.int8, device=dev), torch.empty(1, device=dev)
+    Xq, d = torch.empty((M, K), dtype=torch.int8, device=dev), torch.empty(M, device=dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    wsw = sq.workspace(sq.SQ_OP_SMOOTH_QUANT_WEIGHT, 0, N, K, dev)
+    wsg = sq.workspace(sq.SQ_OP_INT8_GEMM_DEQUANT, M, N, K, dev)
+    Wq1, e1 = torch.empty((N, K), dtype=torch.int8, device=dev), torch.empty(N, device=dev)
+    sq.sq_smooth_quant_weight(W, None, sq.SQ_PER_CHANNEL, Wq1, e1)
+    Y1 = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    wsl = sq.workspace(sq.SQ_OP_LLMINT8, M, N, K, dev)
+
+    def smoothquant():
+        sq.sq_act_channel_absmax(X, amax)
+        sq.sq_smooth_scale(amax, W, p.alpha, s, inv_s)
+        sq.sq_smooth_quant_weight(W, s, sq.SQ_PER_TENSOR, Wq, e, wsw)
+        sq.sq_quant_act_per_token(X, inv_s, Xq, d)
+        sq.sq_int8_gemm_dequant(Xq, Wq, d, e, sq.SQ_PER_TENSOR, None, Y, None, wsg)
+
+    def llmint8():
+        sq.llmint8_decomposed_linear(X, W, Wq1, e1, p.threshold, None, Y1, None, None, None, wsl)
+
+    out = {}
+    for name, fn in (("smoothquant_path", smoothquant), ("llmint8_linear", llmint8)):
+        stream = torch.cuda.current_stream()
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        lat = []
+        for _ in range(50):
+            t0 = time.perf_counter()
+            fn()
+            stream.synchronize()
+            lat.append((time.perf_counter() - t0) * 1e6)
+        out[name] = {"eager_launch_to_result_us": round(statistics.median(lat), 2),
+                     "graph_device_us": round(_graph_time_us(torch, [fn], 20), 2)}
+    out["config"] = f"tiny X[{M},{K}] W[{N},{K}]; SmoothQuant alpha {p.alpha} per-tensor weight; LLM.int8 6.0"
+    return out
+
+
+def measure_kernel_times(path, steps=4):
+    """Device time of every kernel of the step, from the CUDA profiler's activity records
+    (torch.profiler over `steps` untimed steps): the library launches several kernels inside
+    one call (the LLM.int8 linear: column absmax, outlier mask, masked quantization with the
+    gathers, GEMM), which CUDA events around the calls cannot separate."""
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        for i in range(steps):
+            path.step(i)
+        torch.cuda.synchronize()
+    out = {}
+    for ev in prof.key_averages():
+        if getattr(ev, "device_type", None) != torch.autograd.DeviceType.CUDA:
+            continue
+        t = getattr(ev, "self_device_time_total", None) or getattr(ev, "self_cuda_time_total", 0.0)
+        key = ev.key.replace("(anonymous namespace)::", "").replace("unnamed>::", "").replace("void ", "")
+        key = key.split("(")[0].replace("sq::", "")
+        out[key] = {"launches_per_step": ev.count / steps, "avg_us": round(t / max(ev.count, 1), 2)}
     return out
 
 

@@ -33,7 +33,11 @@
  *   - Arguments are validated before anything is launched; a violation returns
  *     SQ_ERR_INVALID / SQ_ERR_ALIGN / SQ_ERR_WORKSPACE, launches nothing and leaves
  *     outputs untouched. sq_last_error() then gives a message (thread-local).
- *   - NaN or Inf inputs are outside the contract (outputs undefined, no error).
+ *   - NaN or Inf inputs are outside the contract (outputs undefined, no error). What the
+ *     kernels happen to produce is not a guarantee: a NaN inside a row quantized by its
+ *     own maximum (per token, per channel) currently gets code -1, one in a row whose
+ *     factor 127/absmax overflowed, or under a per-tensor or clipped scale, gets -128, and
+ *     one under the zero-point form gets the row's zero point (maxima ignore NaNs).
  *   - Rounding: codes use round-half-to-even of (value * (127/absmax)) in fp32 and are
  *     clamped to [-128, 127]; absmax == 0 gives codes 0 and scale 0. The reciprocal
  *     127/absmax and the scale absmax/127 are IEEE fp32 divisions.
@@ -85,8 +89,9 @@ typedef enum {
  *   amax[j] = max_m |X[m, j]|                  (accumulate == 0)
  *   amax[j] = max(amax[j], max_m |X[m, j]|)    (accumulate != 0: running maximum
  *                                               over calibration batches)
- * [SQ] §3.2 (forward hook: x.abs().amax over the token dimensions, torch.maximum
- * across batches); [LLMINT8] §2.1 step 1 (column-wise absolute maximum).
+ * [SQ] §3.2 (a forward hook records each input channel's absolute maximum over the token
+ * dimensions and keeps the running maximum across calibration batches); [LLMINT8] §2.1
+ * step 1 (column-wise absolute maximum).
  * X: bf16 [M, K], ldx. amax: fp32 [K], read (accumulate) and written. Exact (a max).
  */
 SQ_API sq_status sq_act_channel_absmax(const void* X_bf16, int64_t M, int64_t K, int64_t ldx, float* amax,
@@ -123,8 +128,8 @@ SQ_API sq_status sq_smooth_quant_weight(const void* W_bf16, int64_t N, int64_t K
 
 /*
  * Smoothing + per-token dynamic activation quantization in one pass over X.
- * [BASICS] per-token granularity and quantization-flow example (X_scale =
- * X.abs().max(dim=-1)/127); [SQ] §2.3 and §3.4 (divide by s before quantizing,
+ * [BASICS] per-token granularity and quantization-flow example (each token row's scale is
+ * its absolute maximum over 127); [SQ] §2.3 and §3.4 (divide by s before quantizing,
  * fused into one light kernel), here as a multiply by inv_s:
  *   x'[m,k] = X[m,k] * inv_s[k]   (fp32; inv_s == NULL means 1)
  *   a_m = max_k |x'[m,k]|, x_scale[m] = a_m/127, Xq[m,k] = clamp(rne(x' * (127/a_m)), -128, 127)
@@ -192,8 +197,9 @@ SQ_API sq_status llmint8_decomposed_linear(const void* X_bf16, const void* W_bf1
  * global maximum there; the per-channel form needs none). Every GPU that loads the library
  * holds those bytes until the process exits. A shape that would need more scratch than the
  * array holds is rejected with SQ_ERR_WORKSPACE and a message naming both sizes.
- * Set-up: the first call on each device looks the array's device address up (with that
- * device current); make that first call before any stream capture.
+ * Set-up: every call looks the array's device address up on the current device (a host-side
+ * query, so no address outlives a device reset); the first call on a device may load the
+ * library's device code, so make that first call before any stream capture.
  * Concurrency: all calls share the array and it keeps the last call's contents; each
  * per-tensor call resets the maximum it needs before use, but calls that overlap on the GPU
  * (different streams, or several host threads) race on it and must be serialised.
@@ -210,8 +216,9 @@ SQ_API sq_status sq_smooth_quant_weight_noalloc(const void* W_bf16, int64_t N, i
  * the conventions above. */
 
 /*
- * Per-tensor activation quantization. [SQ] §3.4 SmoothQuantLinear.forward (x_max =
- * x.abs().max() over the whole tensor, x_scale = x_max/127, round().clamp(-128, 127)):
+ * Per-tensor activation quantization. [SQ] §3.4 (the reference module scales activations by
+ * one maximum over the whole tensor): a = max |x'| over all elements, scale a/127, codes
+ * clamp(rne(x' * 127/a), -128, 127):
  *   x'[m,k] = X[m,k] * inv_s[k]     (fp32; inv_s == NULL means 1)
  *   a = *clip when clip != NULL (a static calibration value, e.g. from sq_act_abs_percentile;
  *       values beyond it saturate at the clamp), else max |x'| over the tensor

@@ -23,7 +23,7 @@
  *   - quantize by multiplying with a once-per-row fp32 reciprocal r = 127/absmax
  *     ([LLMINT8] §2.2 quantize), dequant scale d = absmax/127 ([BASICS] symmetric
  *     quantization), clamp to [-128,127] ([BASICS] quantization-flow example);
- *   - round half to even (torch.round in [BASICS] quantization-flow example);
+ *   - round half to even (the rounding of the [BASICS] quantization-flow example);
  *   - absmax == 0 gives r = 0, codes 0 and scale 0;
  *   - smoothed values x*inv_s and w*s stay in fp32, never rounded to 16 bits;
  *   - the smoothing factor is s_j = max(a_j,1e-8)^alpha / max(w_j,1e-8)^(1-alpha)
@@ -92,8 +92,9 @@ static int8_t round_clamp_int8(float v) {
 
 /* Per-column absmax of X [M,K] (leading dimension ldx):
  * amax_j = max_m |X[m,j]|, or max(amax_j, .) when accumulate != 0.
- * [SQ] §3.2 calibration hook (x.abs().amax over the token dims, running maximum
- * across batches); [LLMINT8] §2.1 step 1 (column-wise absolute maximum). */
+ * [SQ] §3.2 calibration hook (each input channel's absolute maximum over the token
+ * dimensions, running maximum across batches); [LLMINT8] §2.1 step 1 (column-wise
+ * absolute maximum). */
 void oracle_act_channel_absmax(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,
                                float *amax, int accumulate) {
 #pragma omp parallel for schedule(static)
@@ -141,9 +142,9 @@ static void quantize_with_absmax(const float *v, int64_t n, float a, int8_t *q) 
 }
 
 /* Weight smoothing + quantization, [BASICS] per-tensor / per-channel granularity
- * and quantization-flow example (W_scale = max|W|/127, W_int8 =
- * round(W/W_scale).clamp(-128,127)); [SQ] §3.3 (W' = W * s broadcast over the
- * input dimension) and §3.4 (w_scale = w_max/127).
+ * and quantization-flow example (the scale is the absolute maximum over 127; codes are
+ * rounded and clamped to [-128, 127]); [SQ] §3.3 (each input channel of the weight
+ * multiplied by its s) and §3.4 (weight scale = weight maximum over 127).
  *   w'_{nk} = W[n,k] * s_k  (fp32; s == NULL means s_k = 1)
  *   per-channel: a_n = max_k |w'_{nk}|, e_n = a_n/127, q = clamp(rne(w' * (127/a_n)))
  *   per-tensor : a   = max_{n,k} |w'|,  e_0 = a/127,   likewise. */
@@ -182,8 +183,8 @@ void oracle_smooth_quant_weight(const uint16_t *W, int64_t N, int64_t K, int64_t
 }
 
 /* Per-token dynamic activation quantization, [BASICS] per-token granularity and
- * quantization-flow example (X_scale = X.abs().max(dim=-1)/127); [SQ] §3.4
- * (x = x / scale before quantizing, here as x * inv_s).
+ * quantization-flow example (each token row's scale is its absolute maximum over 127);
+ * [SQ] §3.4 (activations divided by s before quantizing, here as x * inv_s).
  *   x'_{mk} = X[m,k] * inv_s_k  (inv_s == NULL means 1)
  *   a_m = max over k not in skip of |x'_{mk}|, d_m = a_m/127,
  *   q_{mk} = clamp(rne(x'_{mk} * (127/a_m))), and q = 0 where bit k of skip is set.
@@ -304,8 +305,8 @@ void oracle_outlier_product(const uint16_t *X, int64_t ldx, const uint16_t *W, i
 
 /* ------------------------------------------------------------------ variants */
 
-/* Per-tensor activation quantization, [SQ] §3.4 SmoothQuantLinear.forward
- * (x_max = x.abs().max(); x_scale = x_max/127; round(x/x_scale).clamp(-128,127)):
+/* Per-tensor activation quantization, [SQ] §3.4 (the reference module's activation scale is one
+ * maximum over the whole tensor, divided by 127; codes rounded half to even and clamped):
  *   x' = X * inv_s (inv_s NULL: 1); a = clip if clip >= 0 (static calibration, e.g. a
  *   percentile), else max over all |x'|; x_scale[0] = a/127; q = clamp(rne(x' * (127/a))). */
 void oracle_quant_act_per_tensor(const uint16_t *X, int64_t M, int64_t K, int64_t ldx,

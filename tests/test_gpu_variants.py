@@ -243,6 +243,40 @@ def test_norm_smooth_quant(M, K, norm, beta, smooth):
     assert np.array_equal(host(Xq), cq)
 
 
+@pytest.mark.parametrize("K", [4096, 16384])
+@pytest.mark.parametrize("norm", [sq.SQ_NORM_LAYER, sq.SQ_NORM_RMS])
+@pytest.mark.parametrize("eps", [1e-5, 0.0])
+def test_norm_statistics_of_nearly_constant_rows(K, norm, eps):
+    """Rows whose mean is large next to their spread, where a one-pass variance
+    E[x^2] - mean^2 cancels: one repeated value, or a constant 1024 (or 3e4, or 2^100) with
+    one, a few or half of the elements one bf16 step away. The statistics stay within one
+    fp32 ulp of the two-pass definition (rows of one value: the variance is exactly 0, so
+    rstd = 1/sqrt(eps), infinite at eps = 0 for LayerNorm), and the codes follow them."""
+    rng = np.random.default_rng(K + norm)
+    rows = []
+    for base in (1024.0, 3.0e4, 2.0 ** 100, -7.5):
+        step = float(np.spacing(np.float32(base))) * 2 ** 16  # one bf16 step at this magnitude
+        for nd in (0, 1, 3, K // 2):
+            x = np.full(K, base, np.float32)
+            idx = rng.choice(K, nd, replace=False)
+            x[idx] += rng.choice([-1.0, 1.0], nd).astype(np.float32) * np.float32(step)
+            rows.append(x)
+    X = wl.f32_to_bf16_bits(np.stack(rows))
+    M = X.shape[0]
+    g = wl.f32_to_bf16_bits(rng.uniform(0.5, 1.5, K).astype(np.float32))
+    Xq, d, st = empty((M, K), torch.int8), empty(M, torch.float32), empty((M, 2), torch.float32)
+    sq.sq_norm_smooth_quant(dev_bf16(X), norm, dev_bf16(g), None, eps, None, Xq, d, st)
+    sq.sq_sync_status()
+    _, _, _, ost = oracle.norm_smooth_quant(X, norm, g, None, eps, None, with_stats=True)
+    gst = host(st)
+    both_inf = np.isinf(gst) & np.isinf(ost) & (np.sign(gst) == np.sign(ost))
+    assert (_ulps(gst, ost)[~both_inf] <= 1).all(), (gst, ost)
+    finite = np.isfinite(gst).all(axis=1)
+    cq, cd, _ = oracle.norm_smooth_quant(X, norm, g, None, eps, None, stats=gst)
+    assert np.array_equal(host(d)[finite], cd[finite])
+    assert np.array_equal(host(Xq)[finite], cq[finite])
+
+
 # --------------------------------------------------------------------------- mu + k sigma
 def test_three_sigma_example_through_llmint8():
     """从自动驾驶芯片到大语言模型INT8量化训练实战解析 §2.1 example ((2,128,4096) activations

@@ -2,7 +2,8 @@
 device memory (components inside a host engine or plugin interface that owns the device
 memory plan, services that fix their footprint at start-up). Its scratch lives in a static
 device array inside the library; this checks through the C ABI that two calls in a row give
-exactly what sq_smooth_quant_weight gives with a caller-provided workspace.
+exactly what sq_smooth_quant_weight gives with a caller-provided workspace, and exactly the
+oracle's codes and scales.
 
 This file is collected last on purpose, and passes both alone and after the other tests."""
 import ctypes as C
@@ -11,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from w8a8_quantized_gemm_b200 import sq
 from w8a8_quantized_gemm_b200 import workloads as wl
 
@@ -52,6 +54,11 @@ def test_noalloc_matches_workspace_version_two_calls(gran):
         sq.sq_sync_status()
         assert torch.equal(got_q, ref_q)  # integer codes: bit for bit
         assert torch.equal(got_e, ref_e)  # scales: bit for bit (same fp32 operations)
+        # and against the oracle on the same bf16 weight and factors
+        w_bits = W.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+        o_q, o_e = oracle.smooth_quant_weight(w_bits, s.cpu().numpy(), gran)
+        assert np.array_equal(got_q.cpu().numpy(), o_q)
+        assert np.array_equal(got_e.cpu().numpy(), o_e)
 
 
 def test_noalloc_rejects_bad_arguments_without_launch():

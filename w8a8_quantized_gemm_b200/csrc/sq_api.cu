@@ -16,16 +16,12 @@ namespace sq {
 // Per-device error word set by kernels whose bounded waits give up.
 __device__ unsigned int g_status_word;
 
+// Looked up on every launch (a host-side query on the current device): no address is kept
+// across calls, so none outlives a device reset and concurrent host threads share no state.
 unsigned int* device_status_word() {
-  static unsigned int* addr[64] = {nullptr};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return nullptr;
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status_word) == cudaSuccess) addr[dev] = static_cast<unsigned int*>(p);
-  }
-  return addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+  return static_cast<unsigned int*>(p);
 }
 
 namespace {
@@ -249,6 +245,7 @@ sq_status gemm_impl(const char* fn, const int8_t* Xq, const int8_t* Wq, const fl
     g_arm_limit_ns = 0;
     g_arm_fault = 0;
   }
+  if (sq::device_status_word() == nullptr) return fail(SQ_ERR_CUDA, "%s: device status word not found", fn);
   const char* why = "kernel launch";
   cudaError_t e = sq::launch_gemm(a, reinterpret_cast<cudaStream_t>(stream), &why);
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, why);
@@ -281,6 +278,7 @@ sq_status llm_impl(const char* fn, const void* X_bf16, const void* W_bf16, const
                 ws == nullptr ? size_t(0) : ws_bytes);
   if (!aligned16(ws)) return fail(SQ_ERR_ALIGN, "%s: ws not 16-byte aligned", fn);
 
+  if (sq::device_status_word() == nullptr) return fail(SQ_ERR_CUDA, "%s: device status word not found", fn);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const uint16_t* X = static_cast<const uint16_t*>(X_bf16);
   const uint16_t* W = static_cast<const uint16_t*>(W_bf16);

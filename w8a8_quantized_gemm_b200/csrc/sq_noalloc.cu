@@ -11,7 +11,6 @@
 #include "sq_internal.h"
 
 #include <cstdio>
-#include <mutex>
 
 namespace {
 
@@ -21,33 +20,20 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = 256;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mu;
-void* g_scratch_addr[kMaxDevices] = {nullptr};
-
 // Device address of the scratch on the current device. In host code the array's name is
-// only a host-side stand-in, so the address is looked up once per device (with that
-// device current) and cached.
+// only a host-side stand-in, so the address is looked up with the device current. The
+// lookup is a host-side query and is repeated on every call: an address kept from an
+// earlier call would point into freed memory after the program reset the device.
 sq_status scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess)
-    return static_cast<sq_status>(sq::record_error(SQ_ERR_CUDA, "sq_smooth_quant_weight_noalloc: cudaGetDevice failed"));
-  if (dev < 0 || dev >= kMaxDevices)
-    return static_cast<sq_status>(sq::record_error(SQ_ERR_UNSUPPORTED, "sq_smooth_quant_weight_noalloc: device index out of range"));
-  std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr) {
-      char msg[256];
-      snprintf(msg, sizeof msg, "sq_smooth_quant_weight_noalloc: cudaGetSymbolAddress failed: %s",
-               cudaGetErrorString(e));
-      return static_cast<sq_status>(sq::record_error(SQ_ERR_CUDA, msg));
-    }
-    g_scratch_addr[dev] = p;
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || p == nullptr) {
+    char msg[256];
+    snprintf(msg, sizeof msg, "sq_smooth_quant_weight_noalloc: cudaGetSymbolAddress failed: %s",
+             cudaGetErrorString(e));
+    return static_cast<sq_status>(sq::record_error(SQ_ERR_CUDA, msg));
   }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return SQ_OK;
 }
 

@@ -1,7 +1,7 @@
 """Small, self-contained launches of single kernels for profiler captures (ncu).
 
 Usage: python -m w8a8_quantized_gemm_b200.profile_cases
-       {gemm,decode,decode1,llm,quant,absmax,norm,asym,meanstd,percentile,rowsums,gemm_asym}
+       {gemm,decode,decode1,llm,quant,absmax,smooth,wquant,norm,asym,meanstd,percentile,rowsums,gemm_asym}
 
 Each case makes random device inputs of one workload's shape and calls one entry point three
 times (so that a capture can skip the first, cold launch):
@@ -11,6 +11,8 @@ times (so that a capture can skip the first, cold launch):
   llm     llmint8_decomposed_linear, 2048 x 11008 x 4096 with 4 outlier columns (CTA pairs)
   quant   sq_quant_act_per_token with smoothing, X bf16 [8192, 8192] (inputs larger than L2)
   absmax  sq_act_channel_absmax, X bf16 [8192, 8192]
+  smooth  sq_smooth_scale (column maxima of W and the factors in one pass), W bf16 [28672, 8192]
+  wquant  sq_smooth_quant_weight, smoothed, per channel, W bf16 [28672, 8192]
   norm    sq_norm_smooth_quant (LayerNorm with beta, smoothing), X bf16 [8192, 8192]
   asym    sq_quant_act_per_token_asym with smoothing, X bf16 [8192, 8192]
   meanstd sq_act_mean_std_threshold (k = 6), X bf16 [8192, 8192]
@@ -85,6 +87,22 @@ def main(mode: str) -> None:
             else:
                 out = torch.empty(1, device=dev)
                 sq.sq_act_abs_percentile(X, 99.99, out, sq.workspace(sq.SQ_OP_ABS_PERCENTILE, M, 0, K))
+    elif mode in ("smooth", "wquant"):
+        # the 70B-shaped weight W [28672, 8192] (470 MB): the smoothing factors (column maxima of
+        # W in the same pass) or the smoothed per-channel weight quantization (470 -> 235 MB)
+        N, K = 28672, 8192
+        W = (torch.randn(N, K, device=dev) * 0.01).to(torch.bfloat16)
+        amax = torch.rand(K, device=dev) * 10.0
+        s = torch.empty(K, device=dev)
+        inv = torch.empty(K, device=dev)
+        sq.sq_smooth_scale(amax, W, 0.5, s, inv)
+        Wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+        e = torch.empty(N, device=dev)
+        for _ in range(3):
+            if mode == "smooth":
+                sq.sq_smooth_scale(amax, W, 0.5, s, inv)
+            else:
+                sq.sq_smooth_quant_weight(W, s, sq.SQ_PER_CHANNEL, Wq, e)
     elif mode == "rowsums":
         Wq = torch.randint(-127, 128, (28672, 8192), dtype=torch.int8, device=dev)
         rs = torch.empty(28672, dtype=torch.int32, device=dev)

@@ -216,7 +216,11 @@ def test_asymmetric_linear_end_to_end():
 
 
 # --------------------------------------------------------------------------- fused norm
-NORM_SHAPES = [(1, 16), (7, 256), (33, 528), (300, 4096), (9, 8192), (3, 16384)]
+# register rows up to K = 8192 (LayerNorm) / 4096 (RMSNorm), bulk-staged row groups beyond
+# (ragged last chunks at 1040, 2064, 5008 and 12304 columns; more rows than row groups at
+# 700 x 8192 and 1300 x 16384, so every ring slot is refilled several times)
+NORM_SHAPES = [(1, 16), (7, 256), (33, 528), (300, 4096), (9, 8192), (3, 16384), (5, 1040), (37, 2064),
+               (11, 5008), (6, 12304), (1000, 4096), (700, 8192), (1300, 16384)]
 
 
 @pytest.mark.parametrize("M,K", NORM_SHAPES)

@@ -112,6 +112,20 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* gmem, uint32_t byte
                : "memory");
 }
 
+// Contiguous bulk copy global -> shared (this CTA) of `bytes` bytes (16-byte aligned
+// addresses, size a multiple of 16), completion counted on an mbarrier of this CTA.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Named barrier `id` (1..15) over `threads` threads (a multiple of 32) of this CTA.
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // 2-D tiled bulk tensor store shared (this CTA) -> global, tracked by bulk groups.
 // Coordinates must be non-negative; out-of-range parts of the box are not written.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {

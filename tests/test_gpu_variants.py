@@ -80,6 +80,23 @@ def test_abs_percentile_exact(M, K, ld, p):
     assert host(out)[0] == oracle.abs_percentile(np.ascontiguousarray(full[:, :K]), p)
 
 
+def test_statistics_workspaces_serve_calls_in_a_row():
+    """One workspace (sized for the largest call) serves percentile and threshold calls of
+    different shapes in a row, each matching the oracle: nothing a call leaves in the
+    workspace changes the next call's result."""
+    wsp = sq.workspace(sq.SQ_OP_ABS_PERCENTILE, 1, 0, 16)
+    wms = sq.workspace(sq.SQ_OP_MEAN_STD_THRESHOLD, 4096, 0, 64)
+    thr, out = empty(1, torch.float32), empty(1, torch.float32)
+    for M, K, p in [(256, 4096, 99.99), (9, 48, 50.0), (2000, 1024, 0.0), (3, 16, 100.0), (256, 4096, 99.9)]:
+        X = _x(M, K, M + 3 * K)
+        Xt = dev_bf16(X)
+        sq.sq_act_abs_percentile(Xt, p, out, wsp)
+        sq.sq_act_mean_std_threshold(Xt, 6.0, thr, None, wms)
+        sq.sq_sync_status()
+        assert host(out)[0] == oracle.abs_percentile(X, p)
+        assert _ulps(host(thr), oracle.mean_std_threshold(X, 6.0)[0]).max() <= 1
+
+
 def test_smooth_scale_normalised():
     rng = np.random.default_rng(5)
     K, N = 1040, 96

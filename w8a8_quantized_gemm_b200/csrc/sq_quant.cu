@@ -83,6 +83,35 @@ quant_rows_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
   const int64_t step = static_cast<int64_t>(TPR) * 16;
   const int64_t row_stride = static_cast<int64_t>(gridDim.x) * kGroups;
 
+  if constexpr (OUTLIERS) {
+    if (ov.w_src != nullptr) {
+      // the weight's outlier columns first, spread over every CTA (weight row r goes to CTA
+      // r % grid, so each CTA's first few threads take one row each and the scattered loads
+      // overlap the activation rows' streams): w_gathered[r, c] = w[r, idx[c]] for c < count,
+      // 0 up to the next multiple of 64, eight columns (16 bytes) per store
+      const int32_t cnt = __ldg(ov.count);
+      const int32_t padded = (cnt + 63) & ~63;
+      for (int64_t r = static_cast<int64_t>(threadIdx.x) * gridDim.x + blockIdx.x; padded > 0 && r < ov.w_rows;
+           r += static_cast<int64_t>(gridDim.x) * kThreads) {
+        const uint16_t* srow = ov.w_src + r * ov.w_ld;
+        uint4* drow = reinterpret_cast<uint4*>(ov.w_gathered + r * ov.ld_gathered);
+        for (int32_t c0 = 0; c0 < padded; c0 += 8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int32_t c = c0 + 2 * i;
+            const int32_t jl = c < cnt ? __ldg(ov.idx + c) : 0;
+            const int32_t jh = c + 1 < cnt ? __ldg(ov.idx + c + 1) : 0;
+            const uint32_t lo = (c < cnt && SQ_GUARD(jl >= 0 && jl < ov.w_ld)) ? srow[jl] : 0u;
+            const uint32_t hi = (c + 1 < cnt && SQ_GUARD(jh >= 0 && jh < ov.w_ld)) ? srow[jh] : 0u;
+            w[i] = lo | (hi << 16);
+          }
+          if (SQ_GUARD(c0 + 8 <= ov.ld_gathered)) drow[c0 / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+  }
+
   float vs[kVC][16];
   if constexpr (HAS_VEC && !TWO_PASS) {
 #pragma unroll
@@ -270,32 +299,7 @@ quant_rows_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
       }
     }
   }
-  if constexpr (OUTLIERS) {
-    if (ov.w_src != nullptr) {
-      // the weight's outlier columns, one thread per weight row: w_gathered[r, c] = w[r, idx[c]]
-      // for c < count, 0 up to the next multiple of 64, eight columns (16 bytes) per store
-      const int32_t cnt = __ldg(ov.count);
-      const int32_t padded = (cnt + 63) & ~63;
-      for (int64_t r = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; r < ov.w_rows;
-           r += static_cast<int64_t>(gridDim.x) * kThreads) {
-        const uint16_t* srow = ov.w_src + r * ov.w_ld;
-        uint4* drow = reinterpret_cast<uint4*>(ov.w_gathered + r * ov.ld_gathered);
-        for (int32_t c0 = 0; c0 < padded; c0 += 8) {
-          uint32_t w[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int32_t c = c0 + 2 * i;
-            const int32_t jl = c < cnt ? __ldg(ov.idx + c) : 0;
-            const int32_t jh = c + 1 < cnt ? __ldg(ov.idx + c + 1) : 0;
-            const uint32_t lo = (c < cnt && SQ_GUARD(jl >= 0 && jl < ov.w_ld)) ? srow[jl] : 0u;
-            const uint32_t hi = (c + 1 < cnt && SQ_GUARD(jh >= 0 && jh < ov.w_ld)) ? srow[jh] : 0u;
-            w[i] = lo | (hi << 16);
-          }
-          if (SQ_GUARD(c0 + 8 <= ov.ld_gathered)) drow[c0 / 8] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      }
-    }
-  }
+
 }
 
 int num_sms() {

@@ -85,28 +85,27 @@ quant_rows_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
 
   if constexpr (OUTLIERS) {
     if (ov.w_src != nullptr) {
-      // the weight's outlier columns first, spread over every CTA (weight row r goes to CTA
-      // r % grid, so each CTA's first few threads take one row each and the scattered loads
-      // overlap the activation rows' streams): w_gathered[r, c] = w[r, idx[c]] for c < count,
-      // 0 up to the next multiple of 64, eight columns (16 bytes) per store
+      // the weight's outlier columns first, a warp per weight row, spread over every CTA
+      // (warp w of CTA b takes rows b + w * grid, then every grid * warps rows):
+      // w_gathered[r, c] = w[r, idx[c]] for c < count, 0 up to the next multiple of 64. Lane
+      // l gathers the column pair (2l, 2l + 1) of each 64-column block: its loads of the
+      // scattered weight values are independent, so a row costs about one memory round trip,
+      // and the warp stores 128 contiguous bytes per block.
       const int32_t cnt = __ldg(ov.count);
       const int32_t padded = (cnt + 63) & ~63;
-      for (int64_t r = static_cast<int64_t>(threadIdx.x) * gridDim.x + blockIdx.x; padded > 0 && r < ov.w_rows;
-           r += static_cast<int64_t>(gridDim.x) * kThreads) {
+      const int lane = threadIdx.x & 31;
+      constexpr int kWarpsPerCta = kThreads / 32;
+      for (int64_t r = static_cast<int64_t>(threadIdx.x >> 5) * gridDim.x + blockIdx.x; padded > 0 && r < ov.w_rows;
+           r += static_cast<int64_t>(gridDim.x) * kWarpsPerCta) {
         const uint16_t* srow = ov.w_src + r * ov.w_ld;
-        uint4* drow = reinterpret_cast<uint4*>(ov.w_gathered + r * ov.ld_gathered);
-        for (int32_t c0 = 0; c0 < padded; c0 += 8) {
-          uint32_t w[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int32_t c = c0 + 2 * i;
-            const int32_t jl = c < cnt ? __ldg(ov.idx + c) : 0;
-            const int32_t jh = c + 1 < cnt ? __ldg(ov.idx + c + 1) : 0;
-            const uint32_t lo = (c < cnt && SQ_GUARD(jl >= 0 && jl < ov.w_ld)) ? srow[jl] : 0u;
-            const uint32_t hi = (c + 1 < cnt && SQ_GUARD(jh >= 0 && jh < ov.w_ld)) ? srow[jh] : 0u;
-            w[i] = lo | (hi << 16);
-          }
-          if (SQ_GUARD(c0 + 8 <= ov.ld_gathered)) drow[c0 / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+        uint32_t* drow = reinterpret_cast<uint32_t*>(ov.w_gathered + r * ov.ld_gathered);
+        for (int32_t c0 = 0; c0 < padded; c0 += 64) {
+          const int32_t c = c0 + 2 * lane;
+          const int32_t jl = c < cnt ? __ldg(ov.idx + c) : 0;
+          const int32_t jh = c + 1 < cnt ? __ldg(ov.idx + c + 1) : 0;
+          const uint32_t lo = (c < cnt && SQ_GUARD(jl >= 0 && jl < ov.w_ld)) ? srow[jl] : 0u;
+          const uint32_t hi = (c + 1 < cnt && SQ_GUARD(jh >= 0 && jh < ov.w_ld)) ? srow[jh] : 0u;
+          if (SQ_GUARD(c + 2 <= ov.ld_gathered)) drow[c / 2] = lo | (hi << 16);
         }
       }
     }

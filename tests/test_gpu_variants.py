@@ -233,9 +233,9 @@ def test_asymmetric_linear_end_to_end():
 
 
 # --------------------------------------------------------------------------- fused norm
-# register rows up to K = 8192 (LayerNorm) / 4096 (RMSNorm), bulk-staged row groups beyond
-# (ragged last chunks at 1040, 2064, 5008 and 12304 columns; more rows than row groups at
-# 700 x 8192 and 1300 x 16384, so every ring slot is refilled several times)
+# register rows up to K = 4096, pipelined row groups beyond (ragged last chunks at 1040, 2064,
+# 5008 and 12304 columns; a group with a single row at 9 x 8192 and 3 x 16384; more rows than
+# row groups at 700 x 8192 and 1300 x 16384, so every ring slot is refilled several times)
 NORM_SHAPES = [(1, 16), (7, 256), (33, 528), (300, 4096), (9, 8192), (3, 16384), (5, 1040), (37, 2064),
                (11, 5008), (6, 12304), (1000, 4096), (700, 8192), (1300, 16384)]
 

@@ -232,92 +232,99 @@ norm_quant_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int
   }
 }
 
-// Bulk-staged form for long rows (see launch_norm_quant): G row groups of GT threads per CTA, one
-// persistent CTA per SM. Each group streams its rows through a ring of `slots` shared-memory
-// row buffers filled by cp.async.bulk (one thread issues a whole row, completion on the slot's
-// mbarrier), so the number of bytes in flight no longer depends on the registers the
-// arithmetic needs. A thread reads its 8-column chunks (thread t: chunks t, t + GT, ...) from
-// shared memory into registers once, and the slot is handed back to the copy engine right after
-// the row statistics; the values stay in registers through the normalisation and the codes.
-// Same arithmetic as norm_quant_kernel (fp64 statistics in one pass, rounded once to fp32;
-// every later step an IEEE fp32 operation in the same order).
 constexpr int kNormMaxSlots = 6;
 constexpr int kNormSmem = 192 * 1024;  // row ring per CTA
 
+// Row groups for long rows (see launch_norm_quant): G groups of GT threads per CTA, one
+// persistent CTA per SM. Each group streams its rows (row0 + j * stride) through a ring of
+// `slots` shared-memory row buffers filled by cp.async.bulk (one thread issues a whole row,
+// completion on the slot's mbarrier), so the bytes in flight do not depend on the registers
+// the arithmetic needs. A thread owns the 8-column chunks t, t + GT, ... of every row. Each
+// pass of the group's loop works on two rows:
+//   1. the statistics of row j from the warps' partial sums (every warp finishes them itself:
+//      no broadcast, no extra barrier), then row j read from its slot into the normalised,
+//      smoothed values y (kept in registers) and the warp's partial absmax;
+//   2. row j+1 read from its slot into its fp64 partial sums;
+//   3. one group barrier, after which row j's slot goes back to the copy engine, its absmax is
+//      known and its codes are stored.
+// One barrier per row, and the statistics of one row overlap the arithmetic of the previous
+// one; reading each row twice from shared memory keeps no raw row in registers across the
+// barrier. The per-row finish uses a multiply by 1/K and the fp64 reciprocal square root (each
+// within a few fp64 ulps of the divisions and square root written out, far below the fp32
+// rounding of mean_f and rstd_f). Where both operands of an operation are pairs, the fp32 steps
+// use sm_100's packed f32x2 instructions (two IEEE round-to-nearest operations each); the
+// multiply that the beta add follows stays scalar, so that no packed multiply feeds an add (such
+// a pair was observed to execute as one fused multiply-add). The codes use scalar multiplies and
+// adds, each rounded.
 template <int GT, int CH, int G, bool LAYER, bool BETA, bool VEC>
 __global__ void __launch_bounds__(GT * G, 1)
-norm_quant_bulk_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int norm,
+norm_quant_pipe_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
                        const uint16_t* __restrict__ gamma, const uint16_t* __restrict__ beta, float eps,
                        const float* __restrict__ vec, int8_t* __restrict__ q, float* __restrict__ scale,
                        float* __restrict__ mean_rstd, int slots, unsigned int* status, uint64_t wait_limit_ns) {
   constexpr int kWarps = GT / 32;
   extern __shared__ __align__(128) uint8_t ring_all[];
   __shared__ uint64_t full_all[G][kNormMaxSlots];
-  __shared__ double2 red2[G][kWarps];
-  __shared__ float redm[G][kWarps];
-  __shared__ int abort_g[G];  // a wait of the group gave up: the group stops after this row's barrier
-  __shared__ float2 stat_g[G];  // the row's mean_f, rstd_f (from the group's first warp)
+  __shared__ double2 red2[G][2][kWarps];  // partial (sum x, sum x^2) per warp, by row parity
+  __shared__ float redm[G][2][kWarps];    // partial absmax per warp, by row parity
   const int g = threadIdx.x / GT;
   const int t = threadIdx.x % GT;
   const int lane = threadIdx.x & 31;
-  const int wg = t >> 5;  // warp within the group
+  const int wg = t >> 5;
   const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
   uint8_t* ring = ring_all + static_cast<size_t>(g) * slots * row_bytes;
   uint64_t* full = full_all[g];
   if (t == 0) {
     for (int i = 0; i < slots; ++i) mbar_init(full + i, 1);
-    abort_g[g] = 0;
     fence_mbar_init();
   }
   __syncthreads();
   griddep_wait();
   griddep_launch_dependents();
-  (void)norm;
-  constexpr bool layer = LAYER;
-  constexpr bool has_beta = BETA;
-  constexpr bool has_vec = VEC;
-  const int nch = static_cast<int>(K / 8);  // 8-column chunks of a row
+  const int nch = static_cast<int>(K / 8);
   const int64_t stride = static_cast<int64_t>(G) * gridDim.x;
   const int64_t row0 = blockIdx.x + static_cast<int64_t>(g) * gridDim.x;
-  // the group's rows are row0 + j * stride; thread 0 of the group keeps `slots` of them in flight
+  const int64_t nrows = row0 < rows ? (rows - 1 - row0) / stride + 1 : 0;  // this group's rows
+  const double inv_k = 1.0 / static_cast<double>(K);
   int64_t issued = 0;
   if (t == 0) {
-    for (int i = 0; i < slots; ++i) {
-      const int64_t r = row0 + i * stride;
-      if (r >= rows) break;
+    for (int i = 0; i < slots && i < nrows; ++i) {
       mbar_arrive_expect_tx(full + i, row_bytes);
-      bulk_load(ring + static_cast<size_t>(i) * row_bytes, src + r * ld, row_bytes, full + i);
+      bulk_load(ring + static_cast<size_t>(i) * row_bytes, src + (row0 + i * stride) * ld, row_bytes, full + i);
       ++issued;
     }
   }
-  int64_t j = 0;
-  for (int64_t row = row0; row < rows; row += stride, ++j) {
-    const int slot = static_cast<int>(j % slots);
-    // every thread waits for the row; one that gives up still reaches the group barrier below,
-    // where the whole group learns of it and stops together (no thread is left at a barrier)
-    if (!mbar_wait_bounded(full + slot, static_cast<uint32_t>((j / slots) & 1), wait_limit_ns)) {
+
+  int64_t pending = 0;  // the row whose slot was waited for last
+  bool failed = false;  // this thread's wait for a slot gave up
+  auto slot_row = [&](int64_t i) {
+    return reinterpret_cast<const uint4*>(ring + static_cast<size_t>(i % slots) * row_bytes);
+  };
+  // Row i of the group: wait for its slot, read this thread's chunks, leave the warp's partial
+  // sums in red2[g][i & 1]. A thread whose wait gives up still reaches the next group barrier,
+  // which ORs `failed` over the group, so that the whole group stops there together.
+  auto load_stats = [&](int64_t i) {
+    pending = i;
+    if (!mbar_wait_bounded(full + static_cast<int>(i % slots), static_cast<uint32_t>((i / slots) & 1),
+                           wait_limit_ns)) {
       atomicOr(status, kErrProducerWait);
-      abort_g[g] = 1;
+      failed = true;
     }
-    // the row's chunks, from shared memory into registers
-    const uint4* srow = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(slot) * row_bytes);
-    uint4 raw[CH];
-#pragma unroll
-    for (int c = 0; c < CH; ++c) {
-      const int idx = t + c * GT;
-      raw[c] = idx < nch ? srow[idx] : make_uint4(0u, 0u, 0u, 0u);
-    }
-    // statistics in one pass: fp64 sums of x and x^2 (absent columns hold 0)
+    const uint4* srow = slot_row(i);
     double s1a = 0.0, s1b = 0.0, s2a = 0.0, s2b = 0.0;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
-      const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+      const int idx = t + c * GT;
+      const uint4 rc = idx < nch ? srow[idx] : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t w[4] = {rc.x, rc.y, rc.z, rc.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const double xa = static_cast<double>(__uint_as_float(w[i] << 16));
-        const double xb = static_cast<double>(__uint_as_float(w[i] & 0xFFFF0000u));
-        s1a = __dadd_rn(s1a, xa);
-        s1b = __dadd_rn(s1b, xb);
+      for (int k = 0; k < 4; ++k) {
+        const double xa = static_cast<double>(__uint_as_float(w[k] << 16));
+        const double xb = static_cast<double>(__uint_as_float(w[k] & 0xFFFF0000u));
+        if constexpr (LAYER) {
+          s1a = __dadd_rn(s1a, xa);
+          s1b = __dadd_rn(s1b, xb);
+        }
         s2a = __fma_rn(xa, xa, s2a);
         s2b = __fma_rn(xb, xb, s2b);
       }
@@ -325,100 +332,111 @@ norm_quant_bulk_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K
     double s1 = __dadd_rn(s1a, s1b), s2 = __dadd_rn(s2a, s2b);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      s1 = __dadd_rn(s1, __shfl_xor_sync(0xffffffffu, s1, o));
+      if constexpr (LAYER) s1 = __dadd_rn(s1, __shfl_xor_sync(0xffffffffu, s1, o));
       s2 = __dadd_rn(s2, __shfl_xor_sync(0xffffffffu, s2, o));
     }
-    if (lane == 0) red2[g][wg] = make_double2(s1, s2);
-    named_bar_sync(1 + g, GT);  // every thread of the group has read the slot and its partials
-    if (abort_g[g]) break;      // uniform over the group
-    if (t == 0) {
-      // the slot goes back to the copy engine for the group's row `slots` rows ahead
-      const int64_t r = row + static_cast<int64_t>(slots) * stride;
-      if (r < rows) {
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(full + slot, row_bytes);
-        bulk_load(ring + static_cast<size_t>(slot) * row_bytes, src + r * ld, row_bytes, full + slot);
-        ++issued;
-      }
+    if (lane == 0) red2[g][i & 1][wg] = make_double2(s1, s2);
+  };
+  // After the group barrier that follows the last read of row i, its slot takes row i + slots.
+  auto refill = [&](int64_t i) {
+    if (t == 0 && i + slots < nrows) {
+      const int slot = static_cast<int>(i % slots);
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(full + slot, row_bytes);
+      bulk_load(ring + static_cast<size_t>(slot) * row_bytes, src + (row0 + (i + slots) * stride) * ld, row_bytes,
+                full + slot);
+      ++issued;
     }
-    // the group's first warp finishes the statistics (fp64 division and square root once per
-    // row, not once per warp) and hands them to the others through shared memory
-    if (wg == 0) {
-      s1 = red2[g][0].x;
-      s2 = red2[g][0].y;
+  };
+
+  bool aborted = false;
+  if (nrows > 0) {
+    load_stats(0);
+    aborted = named_bar_sync_or(1 + g, GT, failed);
+  }
+  for (int64_t j = 0; j < nrows && !aborted; ++j) {
+    const int p = static_cast<int>(j & 1);
+    // 1. statistics of row j (the same fixed order of the warps' partials in every warp)
+    double s1 = 0.0, s2 = 0.0;
 #pragma unroll
-      for (int w = 1; w < kWarps; ++w) {
-        s1 = __dadd_rn(s1, red2[g][w].x);
-        s2 = __dadd_rn(s2, red2[g][w].y);
-      }
-      const double kd = static_cast<double>(K);
-      float mf = 0.0f;
-      double m2 = __ddiv_rn(s2, kd);
-      if (layer) {
-        const double mean = __ddiv_rn(s1, kd);
-        mf = __double2float_rn(mean);
-        m2 = fmax(__dsub_rn(m2, __dmul_rn(mean, mean)), 0.0);
-      }
-      const float rf = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(m2, static_cast<double>(eps)))));
-      if (lane == 0) stat_g[g] = make_float2(mf, rf);
+    for (int w = 0; w < kWarps; ++w) {
+      const double2 v = red2[g][p][w];
+      if constexpr (LAYER) s1 = __dadd_rn(s1, v.x);
+      s2 = __dadd_rn(s2, v.y);
     }
-    named_bar_sync(1 + g, GT);
-    const float mean_f = stat_g[g].x;
-    const float rstd_f = stat_g[g].y;
-    // y = ((x - mean) * rstd) * gamma + beta, x' = y * inv_s, absmax
-    float xs[CH][8];
+    float mean_f = 0.0f;
+    double m2 = __dmul_rn(s2, inv_k);
+    if constexpr (LAYER) {
+      const double mean = __dmul_rn(s1, inv_k);
+      mean_f = __double2float_rn(mean);
+      m2 = fmax(__dsub_rn(m2, __dmul_rn(mean, mean)), 0.0);
+    }
+    const float rstd_f = __double2float_rn(rsqrt(__dadd_rn(m2, static_cast<double>(eps))));
+    const uint64_t mean2 = f2_pack(mean_f, mean_f);
+    const uint64_t rstd2 = f2_pack(rstd_f, rstd_f);
+    // y = ((x - mean) * rstd) * gamma + beta, x' = y * inv_s; absmax
+    const uint4* srow = slot_row(j);
+    float y[CH][8];
     float a = 0.0f;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int idx = t + c * GT;
-      float gv[8], bv[8], vv[8];
-      const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
       if (idx < nch) {
+        const uint4 rc = srow[idx];
         const uint4 g4 = __ldg(reinterpret_cast<const uint4*>(gamma) + idx);
         const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          gv[2 * i] = __uint_as_float(gw[i] << 16);
-          gv[2 * i + 1] = __uint_as_float(gw[i] & 0xFFFF0000u);
-        }
-        if (has_beta) {
+        uint32_t bw[4] = {0u, 0u, 0u, 0u};
+        if constexpr (BETA) {
           const uint4 b4 = __ldg(reinterpret_cast<const uint4*>(beta) + idx);
-          const uint32_t bw[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            bv[2 * i] = __uint_as_float(bw[i] << 16);
-            bv[2 * i + 1] = __uint_as_float(bw[i] & 0xFFFF0000u);
-          }
+          bw[0] = b4.x; bw[1] = b4.y; bw[2] = b4.z; bw[3] = b4.w;
         }
-        if (has_vec) {
-          const float4 v0 = __ldg(reinterpret_cast<const float4*>(vec) + 2 * idx);
-          const float4 v1 = __ldg(reinterpret_cast<const float4*>(vec) + 2 * idx + 1);
-          vv[0] = v0.x; vv[1] = v0.y; vv[2] = v0.z; vv[3] = v0.w;
-          vv[4] = v1.x; vv[5] = v1.y; vv[6] = v1.z; vv[7] = v1.w;
+        uint64_t vv[4] = {0u, 0u, 0u, 0u};
+        if constexpr (VEC) {
+          const ulonglong2 v0 = __ldg(reinterpret_cast<const ulonglong2*>(vec) + 2 * idx);
+          const ulonglong2 v1 = __ldg(reinterpret_cast<const ulonglong2*>(vec) + 2 * idx + 1);
+          vv[0] = v0.x; vv[1] = v0.y; vv[2] = v1.x; vv[3] = v1.y;
+        }
+        const uint32_t xw[4] = {rc.x, rc.y, rc.z, rc.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint64_t v2 = f2_pack(__uint_as_float(xw[k] << 16), __uint_as_float(xw[k] & 0xFFFF0000u));
+          if constexpr (LAYER) v2 = f2_sub(v2, mean2);
+          v2 = f2_mul(v2, rstd2);
+          float y0, y1;
+          if constexpr (BETA) {
+            f2_unpack(v2, y0, y1);
+            y0 = __fadd_rn(__fmul_rn(y0, __uint_as_float(gw[k] << 16)), __uint_as_float(bw[k] << 16));
+            y1 = __fadd_rn(__fmul_rn(y1, __uint_as_float(gw[k] & 0xFFFF0000u)), __uint_as_float(bw[k] & 0xFFFF0000u));
+            if constexpr (VEC) f2_unpack(f2_mul(f2_pack(y0, y1), vv[k]), y0, y1);
+          } else {
+            v2 = f2_mul(v2, f2_pack(__uint_as_float(gw[k] << 16), __uint_as_float(gw[k] & 0xFFFF0000u)));
+            if constexpr (VEC) v2 = f2_mul(v2, vv[k]);
+            f2_unpack(v2, y0, y1);
+          }
+          y[c][2 * k] = y0;
+          y[c][2 * k + 1] = y1;
+          a = fmaxf(a, fmaxf(fabsf(y0), fabsf(y1)));
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) gv[i] = 0.0f;  // absent columns: y = 0
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float x = (i & 1) ? __uint_as_float(w[i >> 1] & 0xFFFF0000u) : __uint_as_float(w[i >> 1] << 16);
-        float y = layer ? __fmul_rn(__fsub_rn(x, mean_f), rstd_f) : __fmul_rn(x, rstd_f);
-        y = __fmul_rn(y, gv[i]);
-        if (has_beta && idx < nch) y = __fadd_rn(y, bv[i]);
-        if (has_vec && idx < nch) y = __fmul_rn(y, vv[i]);
-        xs[c][i] = y;
-        a = fmaxf(a, fabsf(y));
+        for (int k = 0; k < 8; ++k) y[c][k] = 0.0f;
       }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    if (lane == 0) redm[g][wg] = a;
-    named_bar_sync(1 + g, GT);
-    a = redm[g][0];
+    if (lane == 0) redm[g][p][wg] = a;
+    // 2. the next row
+    if (j + 1 < nrows) load_stats(j + 1);
+    // 3. one barrier: row j's partial maxima and row j+1's partial sums are in, row j's slot
+    //    has been read for the last time by every thread
+    aborted = named_bar_sync_or(1 + g, GT, failed);
+    if (aborted) break;
+    refill(j);
+    a = redm[g][p][0];
 #pragma unroll
-    for (int w = 1; w < kWarps; ++w) a = fmaxf(a, redm[g][w]);
+    for (int w = 1; w < kWarps; ++w) a = fmaxf(a, redm[g][p][w]);
     const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+    const int64_t row = row0 + j * stride;
     if (t == 0) {
       scale[row] = __fdiv_rn(a, 127.0f);
       if (mean_rstd != nullptr) {
@@ -426,31 +444,28 @@ norm_quant_bulk_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K
         mean_rstd[2 * row + 1] = rstd_f;
       }
     }
-    // codes: 8 bytes per chunk; a row scaled by its own maximum needs no clamp unless r
-    // overflowed (a below 127 / FLT_MAX)
+    // codes: a row scaled by its own maximum needs no clamp unless r overflowed
     int8_t* qrow = q + row * K;
     const bool clamp = !(r <= 3.402823466e38f);
-    const uint64_t r2 = f2_pack(r, r);
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int idx = t + c * GT;
       if (idx < nch && SQ_GUARD(idx * 8 + 8 <= K)) {
         int qv[8];
 #pragma unroll
-        for (int i = 0; i < 8; i += 2) {
-          if (clamp)
-            q8x2<true>(xs[c][i], xs[c][i + 1], r2, qv[i], qv[i + 1]);
-          else
-            q8x2<false>(xs[c][i], xs[c][i + 1], r2, qv[i], qv[i + 1]);
+        for (int k = 0; k < 8; ++k) {
+          float tq = __fmul_rn(y[c][k], r);
+          if (clamp) tq = fminf(fmaxf(tq, -128.0f), 127.0f);
+          qv[k] = __float_as_int(__fadd_rn(tq, 12582912.0f));
         }
-        *reinterpret_cast<uint2*>(qrow + idx * 8) = make_uint2(pack4(qv[0], qv[1], qv[2], qv[3]),
-                                                               pack4(qv[4], qv[5], qv[6], qv[7]));
+        *reinterpret_cast<uint2*>(qrow + idx * 8) =
+            make_uint2(pack4(qv[0], qv[1], qv[2], qv[3]), pack4(qv[4], qv[5], qv[6], qv[7]));
       }
     }
   }
-  // copies issued for rows this group did not reach (after a timed-out wait) land before exit
-  if (t == 0) {
-    for (int64_t k = j; k < issued; ++k) {
+  // copies issued for rows this group did not consume (after a timed-out wait) land before exit
+  if (t == 0 && aborted) {
+    for (int64_t k = pending; k < issued; ++k) {
       if (!mbar_wait_bounded(full + static_cast<int>(k % slots), static_cast<uint32_t>((k / slots) & 1),
                              wait_limit_ns))
         atomicOr(status, kErrTeardownWait);
@@ -459,12 +474,14 @@ norm_quant_bulk_kernel(const uint16_t* __restrict__ src, int64_t rows, int64_t K
 }
 
 template <int GT, int CH, int G, bool LAYER, bool BETA, bool VEC>
-cudaError_t launch_norm_bulk_t(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, int norm,
-                               const uint16_t* gamma, const uint16_t* beta, float eps, const float* vec, int8_t* q,
-                               float* scale, float* mean_rstd, cudaStream_t stream) {
-  auto kernel = norm_quant_bulk_kernel<GT, CH, G, LAYER, BETA, VEC>;
+cudaError_t launch_norm_pipe_t(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, const uint16_t* gamma,
+                               const uint16_t* beta, float eps, const float* vec, int8_t* q, float* scale,
+                               float* mean_rstd, cudaStream_t stream) {
+  auto kernel = norm_quant_pipe_kernel<GT, CH, G, LAYER, BETA, VEC>;
   const int64_t row_bytes = K * 2;
   const int slots = static_cast<int>(std::min<int64_t>(kNormMaxSlots, kNormSmem / (G * row_bytes)));
+  // a group holds two rows at once (row j being normalised, row j+1 being summed)
+  if (slots < 2 || K > static_cast<int64_t>(GT) * CH * 8) return cudaErrorInvalidConfiguration;
   const size_t smem = static_cast<size_t>(G) * slots * row_bytes;
   static std::atomic<uint64_t> attr_done{0};  // one bit per device
   int dev = 0;
@@ -479,21 +496,24 @@ cudaError_t launch_norm_bulk_t(const uint16_t* src, int64_t rows, int64_t K, int
   if (status == nullptr) return cudaErrorInvalidSymbol;
   const int64_t blocks = std::min<int64_t>(sm_count(), (rows + G - 1) / G);
   return launch_kernel(kernel, dim3(static_cast<unsigned>(blocks)), dim3(GT * G), smem, stream, false, src, rows, K,
-                       ld, norm, gamma, beta, eps, vec, q, scale, mean_rstd, slots, status, kDefaultWaitLimitNs);
+                       ld, gamma, beta, eps, vec, q, scale, mean_rstd, slots, status, kDefaultWaitLimitNs);
 }
 
-// The norm kind and the presence of beta and of the smoothing vector are compile-time flags
-// of the bulk kernel: no per-element branch or predicate on them.
-template <int GT, int CH, int G, bool LAYER>
-cudaError_t launch_norm_bulk(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, int norm,
+// The norm kind and the presence of beta and of the smoothing vector are compile-time flags.
+template <int GT, int CH, int G>
+cudaError_t launch_norm_pipe(const uint16_t* src, int64_t rows, int64_t K, int64_t ld, int norm,
                              const uint16_t* gamma, const uint16_t* beta, float eps, const float* vec, int8_t* q,
                              float* scale, float* mean_rstd, cudaStream_t stream) {
-#define SQ_BULK(B, V) \
-  launch_norm_bulk_t<GT, CH, G, LAYER, B, V>(src, rows, K, ld, norm, gamma, beta, eps, vec, q, scale, mean_rstd, stream)
+#define SQ_PIPE(L, B, V) \
+  launch_norm_pipe_t<GT, CH, G, L, B, V>(src, rows, K, ld, gamma, beta, eps, vec, q, scale, mean_rstd, stream)
   const bool b = beta != nullptr, v = vec != nullptr;
-  if (b) return v ? SQ_BULK(true, true) : SQ_BULK(true, false);
-  return v ? SQ_BULK(false, true) : SQ_BULK(false, false);
-#undef SQ_BULK
+  if (norm == 0) {
+    if (b) return v ? SQ_PIPE(true, true, true) : SQ_PIPE(true, true, false);
+    return v ? SQ_PIPE(true, false, true) : SQ_PIPE(true, false, false);
+  }
+  if (b) return v ? SQ_PIPE(false, true, true) : SQ_PIPE(false, true, false);
+  return v ? SQ_PIPE(false, false, true) : SQ_PIPE(false, false, false);
+#undef SQ_PIPE
 }
 
 template <int TPR, int CHUNKS>
@@ -696,20 +716,16 @@ cudaError_t launch_norm_quant(const uint16_t* src, int64_t rows, int64_t K, int6
                               const uint16_t* gamma, const uint16_t* beta, float eps, const float* vec, int8_t* q,
                               float* scale, float* mean_rstd, cudaStream_t stream) {
 #define SQ_NORM_ARGS src, rows, K, ld, norm, gamma, beta, eps, vec, q, scale, mean_rstd, stream
-  // Measured on X [M, K] with M = 2048..8192 (graph-timed, one B200): the bulk-staged row
-  // groups win for K > 8192 (LayerNorm 107 vs 117 us, RMSNorm 83 vs 106 us at 4096 x 16384)
-  // and for RMSNorm at 4096 < K <= 8192 (82 vs 89 us at 8192 x 8192); the register rows win
-  // elsewhere (LayerNorm 99 vs 107 us at 8192 x 8192, 26 vs 32 us at 8192 x 2048).
+  // Measured on X [M, K] with M = 2048..8192 (graph-timed, one B200): the pipelined row groups
+  // win for K > 4096 (LayerNorm / RMSNorm 87 / 78 us at 8192 x 8192 against 99 / 82 us for the
+  // best earlier forms, 86 / 80 us against 106 / 82 us at 4096 x 16384); at K <= 4096 they are
+  // no faster than the register rows (13.6 vs 13.7 us at 2048 x 4096).
   if (K <= 512) return launch_norm_t<32, 1>(SQ_NORM_ARGS);
   if (K <= 1024) return launch_norm_t<64, 1>(SQ_NORM_ARGS);
   if (K <= 2048) return launch_norm_t<128, 1>(SQ_NORM_ARGS);
   if (K <= 4096) return launch_norm_t<256, 1>(SQ_NORM_ARGS);
-  if (K <= 8192) {
-    if (norm != 0) return launch_norm_bulk<128, 8, 4, false>(SQ_NORM_ARGS);
-    return launch_norm_t<256, 2>(SQ_NORM_ARGS);
-  }
-  if (norm != 0) return launch_norm_bulk<256, 8, 2, false>(SQ_NORM_ARGS);
-  return launch_norm_bulk<256, 8, 2, true>(SQ_NORM_ARGS);
+  if (K <= 8192) return launch_norm_pipe<128, 8, 4>(SQ_NORM_ARGS);
+  return launch_norm_pipe<256, 8, 2>(SQ_NORM_ARGS);
 #undef SQ_NORM_ARGS
 }
 

@@ -35,9 +35,10 @@ int record_error(int st, const char* msg);
 // still finishing, so its launch and set-up (barrier init, TMEM allocation, descriptor
 // prefetch) overlap that kernel's tail; the wait returns once the previous grid has
 // completed and its writes are visible, so the stream order of the data is unchanged.
-// Only short, latency-bound launches take it: measured on the whole SmoothQuant +
-// LLM.int8 step (2048 x 11008 x 4096), setting it on every launch made the step 1-3%
-// slower, while a 4096 x 4096 decode GEMM gains ~0.8 us (of ~10.6).
+// The GEMM launches and the short, latency-bound launches take it: measured on the whole
+// SmoothQuant + LLM.int8 step (2048 x 11008 x 4096), setting it on every launch made the step
+// 1-3% slower, on the GEMM launches alone about 1% faster, and a 4096 x 4096 decode GEMM gains
+// ~0.8 us (of ~10.6).
 // `cluster_x` > 1 groups consecutive CTAs into clusters of that many (CTA pairs: 2).
 template <typename... KArgs, typename... Args>
 cudaError_t launch_kernel_clustered(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,

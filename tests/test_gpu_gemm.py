@@ -38,11 +38,14 @@ def _gemm_direct(xq, wq, d, e, gran, bias_bits):
 # CTA would only compute padding). Up to 4 tokens take the CUDA-core product (a warp per output
 # channel): (1, 8, 16) gives one CTA fewer channels than warps, (4, 3000, 4096) a channel count
 # that is no multiple of the CTA's warps, (2, 520, 16384) the longest rows (several rounds of
-# loads per row), (3, 2000, 12304) a last round of loads that runs past the end of the row
+# loads per row), (3, 2000, 12304) a last round of loads that runs past the end of the row.
+# More swapped K splits: (33, 4736, 2048) on all 148 SMs (one token in the second column
+# half), (48, 3000, 1024) with a ragged last weight tile, (8, 2048, 4096) in eight parts
 GEMM_SHAPES = [(1, 8, 16), (16, 256, 256), (5, 24, 48), (130, 72, 144), (200, 264, 208), (128, 128, 4096),
                (257, 1000, 528), (3, 200, 1040), (64, 4096, 4096), (1024, 2048, 1024), (300, 9480, 528),
                (2304, 2120, 720), (37, 9736, 256), (1, 4096, 4096), (65, 296, 512), (2433, 1800, 272),
-               (4100, 1288, 1040), (100, 37888, 128), (4, 3000, 4096), (2, 520, 16384), (3, 2000, 12304)]
+               (4100, 1288, 1040), (100, 37888, 128), (4, 3000, 4096), (2, 520, 16384), (3, 2000, 12304),
+               (33, 4736, 2048), (48, 3000, 1024), (8, 2048, 4096)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)

@@ -18,17 +18,6 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-// One lane of the calling warp is elected (returns true there), all lanes must call.
-__device__ __forceinline__ bool elect_one() {
-  uint32_t pred = 0;
-  asm volatile(
-      "{\n\t.reg .pred P;\n\t.reg .b32 R;\n\t"
-      "elect.sync R|P, 0xffffffff;\n\t"
-      "selp.u32 %0, 1, 0, P;\n\t}"
-      : "=r"(pred));
-  return pred != 0;
-}
-
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -121,13 +110,9 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
                : "memory");
 }
 
-// Named barrier `id` (1..15) over `threads` threads (a multiple of 32) of this CTA.
-__device__ __forceinline__ void named_bar_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
-// Named barrier that also ORs one predicate over its `threads` threads: every thread gets
-// the same result, whatever the order in which they arrive.
+// Named barrier `id` (1..15) over `threads` threads (a multiple of 32) of this CTA that also ORs
+// one predicate over them: every thread gets the same result, whatever the order in which they
+// arrive.
 __device__ __forceinline__ bool named_bar_sync_or(int id, int threads, bool v) {
   uint32_t r;
   asm volatile(

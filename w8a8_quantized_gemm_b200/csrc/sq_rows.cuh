@@ -16,15 +16,6 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
   return __byte_perm(ab, cd, 0x5410u);
 }
 
-// clamp(rne(x * r), -128, 127), returned in the low byte (the upper bytes are not the code).
-// The product is clamped first (the same result: every value in [127, 128) rounds to 127 or
-// 128 and clamps to 127, likewise at -128), then rounded half to even by adding 1.5 * 2^23,
-// whose fp32 sum keeps the integer in its low mantissa bits: no float->int conversion unit.
-__device__ __forceinline__ int q8(float x, float r) {
-  const float t = fminf(fmaxf(__fmul_rn(x, r), -128.0f), 127.0f);
-  return __float_as_int(__fadd_rn(t, 12582912.0f));
-}
-
 // Packed pairs of fp32 (sm_100 f32x2 arithmetic: two IEEE round-to-nearest operations per
 // instruction, each lane exactly the scalar result). Use them only where no packed multiply
 // feeds a packed add: such a pair was observed to execute as one fused multiply-add.
@@ -52,8 +43,12 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
   return r;
 }
 
-// q8 of two values at once. With CLAMP the products and the rounding add are packed, and
-// the clamp between them keeps the two from fusing. Without CLAMP the caller guarantees
+// clamp(rne(x * r), -128, 127) of two values, each returned in the low byte (the upper bytes
+// are not the code). The product is clamped first (the same result: every value in [127, 128)
+// rounds to 127 or 128 and clamps to 127, likewise at -128), then rounded half to even by
+// adding 1.5 * 2^23, whose fp32 sum keeps the integer in its low mantissa bits: no float->int
+// conversion unit. With CLAMP the products and the rounding add are packed, and the clamp
+// between them keeps the two from fusing. Without CLAMP the caller guarantees
 // |x * r| < 127.5: a row scaled by r = 127/a with a its own absmax (|x| <= a, r finite) stays
 // within 127 * (1 + 2^-24)^2, which rounds to a code in [-127, 127], so the clamp could not
 // change a code; the products are then scalar multiplies with an explicit rounding mode, which
@@ -147,28 +142,6 @@ __device__ __forceinline__ void widen16(const uint4 (&r)[2], float (&v)[16]) {
     v[2 * i] = __uint_as_float(w[i] << 16);
     v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
-}
-
-// Sum over the TPR threads of one row group in fp64 (fixed order: butterfly within the warp,
-// then the warps of the group in index order); every thread of the group gets the result.
-template <int TPR>
-__device__ __forceinline__ double group_sum(double a, double* red /* [CTA threads / 32] */) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) a = __dadd_rn(a, __shfl_xor_sync(0xffffffffu, a, o));
-  if constexpr (TPR > 32) {
-    constexpr int kWarpsPerGroup = TPR / 32;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int g0 = (warp / kWarpsPerGroup) * kWarpsPerGroup;
-    if (lane == 0) red[warp] = a;
-    __syncthreads();
-    double t = red[g0];
-#pragma unroll
-    for (int w = 1; w < kWarpsPerGroup; ++w) t = __dadd_rn(t, red[g0 + w]);
-    __syncthreads();
-    a = t;
-  }
-  return a;
 }
 
 // Two fp64 sums over the TPR threads of one row group at once (one shared-memory round).

@@ -266,8 +266,9 @@ SQ_API sq_status sq_int8_gemm_dequant_ex(const int8_t* Xq, const int8_t* Wq, con
  * smoothing folded into the output of the LayerNorm that precedes the linear layer
  * ([SQ] §4.2 fuse the scaling into the previous operation's output; §4.5 second detail).
  * Per row m, statistics in fp64 rounded once to fp32 (computed in one pass from the sums of
- * x and x^2; within fp64 rounding of the two-pass form below, so on rare rows a statistic
- * may differ from a two-pass evaluation by one fp32 ulp):
+ * x and x^2; for K > 4096 the division by K is a multiply by 1/K and 1/sqrt a reciprocal
+ * square root, each within a few fp64 ulps; so on rare rows a statistic may differ from a
+ * two-pass evaluation by one fp32 ulp):
  *   SQ_NORM_LAYER: mean = sum_k x / K, var = sum_k (x - mean)^2 / K,
  *                  rstd = fp32(1/sqrt(var + eps)), y = ((x - fp32(mean)) * rstd) * gamma_k + beta_k
  *   SQ_NORM_RMS:   rstd = fp32(1/sqrt(sum_k x^2 / K + eps)),   y = (x * rstd) * gamma_k + beta_k

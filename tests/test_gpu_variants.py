@@ -240,9 +240,15 @@ NORM_SHAPES = [(1, 16), (7, 256), (33, 528), (300, 4096), (9, 8192), (3, 16384),
                (11, 5008), (6, 12304), (1000, 4096), (700, 8192), (1300, 16384)]
 
 
-@pytest.mark.parametrize("M,K", NORM_SHAPES)
+# beta without smoothing and smoothing without beta: the remaining compile-time forms of the
+# pipelined row groups (both group shapes, a ragged row)
+NORM_MIXED = [(M, K, beta, smooth) for (M, K) in [(9, 8192), (700, 8192), (6, 12304), (300, 4096)]
+              for (beta, smooth) in [(True, False), (False, True)]]
+
+
+@pytest.mark.parametrize("M,K,beta,smooth", [(M, K, b, s) for (M, K) in NORM_SHAPES for (b, s) in
+                                             [(True, True), (False, False)]] + NORM_MIXED)
 @pytest.mark.parametrize("norm", [sq.SQ_NORM_LAYER, sq.SQ_NORM_RMS])
-@pytest.mark.parametrize("beta,smooth", [(True, True), (False, False)])
 def test_norm_smooth_quant(M, K, norm, beta, smooth):
     rng = np.random.default_rng(M + K + 10 * norm + 100 * beta)
     X = wl.f32_to_bf16_bits(rng.normal(0.3, 2.0, (M, K)).astype(np.float32))
@@ -264,7 +270,7 @@ def test_norm_smooth_quant(M, K, norm, beta, smooth):
     assert np.array_equal(host(Xq), cq)
 
 
-@pytest.mark.parametrize("K", [4096, 16384])
+@pytest.mark.parametrize("K", [4096, 8192, 16384])
 @pytest.mark.parametrize("norm", [sq.SQ_NORM_LAYER, sq.SQ_NORM_RMS])
 @pytest.mark.parametrize("eps", [1e-5, 0.0])
 def test_norm_statistics_of_nearly_constant_rows(K, norm, eps):

@@ -113,7 +113,7 @@ def test_variant_validation():
                                      None) == sq.SQ_ERR_INVALID
     assert L.sq_int8_gemm_dequant_ex(FAKE, FAKE, FAKE, 5, None, FAKE, 1, None, None, FAKE, 16, 16, 64, None, None, 0,
                                      None) == sq.SQ_ERR_INVALID
-    # fused norm: K above the register-resident limit, bad norm, negative eps, no gamma
+    # fused norm: K above 16384 (the longest row a row group holds), bad norm, negative eps, no gamma
     assert L.sq_norm_smooth_quant(FAKE, 4, 16400, 16400, 0, FAKE, None, C.c_float(1e-5), None, FAKE, FAKE, None,
                                   None) == sq.SQ_ERR_INVALID
     assert L.sq_norm_smooth_quant(FAKE, 4, 64, 64, 2, FAKE, None, C.c_float(1e-5), None, FAKE, FAKE, None,

@@ -3,7 +3,8 @@ pairs and K split each shape gets, read through the sq_debug_gemm_plan hook, aga
 restated here from the kernel design (not from the planner's code):
 
 - up to 4 tokens without outlier columns (K <= 16384): the CUDA-core product;
-- up to 64 tokens without outlier columns: swapped operands, 64-token tiles;
+- up to 64 tokens without outlier columns: swapped operands, 32-token tiles up to 32 tokens and
+  64-token tiles above;
 - otherwise the widest of 256/128/64 whose 128-row tile count covers the 148 SMs;
 - 256-wide tiles run on CTA pairs (256 x 256) when the pair tiles cover the 74 SM pairs and
   the 256-row tiles add no padded rows (an even number of 128-row tiles, or >= 32 of them);
@@ -46,8 +47,8 @@ def test_few_tokens_use_the_cuda_core_product(M):
 @pytest.mark.parametrize("M", [5, 16, 64])
 def test_decode_swaps_and_splits_k(M):
     p = plan(M, 4096, 4096)
-    assert p["path"] == sq.GEMM_PATH_TENSOR and p["swap"] == 1 and p["bn"] == 64
-    tiles = 4096 // 128  # weight rows on the 128-row operand, one 64-token column tile
+    assert p["path"] == sq.GEMM_PATH_TENSOR and p["swap"] == 1 and p["bn"] == (32 if M <= 32 else 64)
+    tiles = 4096 // 128  # weight rows on the 128-row operand, one token column tile
     assert p["whole_tiles"] == 0 and p["split_tiles"] == tiles
     kb = 4096 // 128
     assert p["splits"] >= 2 and p["splits"] * tiles <= SMS

@@ -69,6 +69,11 @@ constexpr int kEpiSmem = kEpiWarps * kEpiBufs * kStageTileBytes;
 // tile i+1, by which time the epilogue has written tile i back, so neither product waits for
 // the other in the common case.
 constexpr int pow2_cols(int c) { return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512; }
+// Bytes of one K-split unit's int32 partial in the workspace: every epilogue warp's 32 rows x 32
+// columns for each chunk of its column half (the larger half when BN / 32 is odd).
+constexpr int64_t split_slot_bytes(int bn) {
+  return static_cast<int64_t>(kEpiWarps) * ((bn / 32 + 1) / 2) * 32 * 32 * 4;
+}
 constexpr int kOutlierLag = 8;
 template <int BN, bool OUTLIERS, int ACC_BUFS, bool PAIR = false>
 struct Cfg {
@@ -115,6 +120,7 @@ struct Params {
   int kb_per_split;
   int32_t* partials;   // [tail tiles * splits][kEpiWarps][BN/64 chunks][8][32 lanes] int4 (int32 x4)
   int32_t* counters;   // [tail tiles * kEpiWarps] arrival counters, zero between calls
+  int64_t partial_int4;  // int4 elements of the partials region (bounds guard)
   const int32_t* o_count;
   // short (programmatic) launches: the weight tiles of the CTA's first work unit are
   // prefetched into L2 before the wait on the previous kernel (the weight does not depend
@@ -880,7 +886,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // the last split of its 32-row x BN/2 sub-tile sums all partials (exact) and stores Y.
         // Partials are stored warp-contiguous (lane-minor), so every access moves 512 bytes.
         const int64_t tail = tile_mn - p.num_full;
-        constexpr int64_t kSlotInt4 = static_cast<int64_t>(kEpiWarps) * kChunks * 8 * 32;
+        constexpr int64_t kSlotInt4 = split_slot_bytes(BN) / 16;
+        static_assert(kSlotInt4 == static_cast<int64_t>(kEpiWarps) * kChunks * 8 * 32, "slot layout");
         auto part_ptr = [&](int sidx, int c) {
           return reinterpret_cast<int4*>(p.partials) + (tail * p.splits + sidx) * kSlotInt4 +
                  ((static_cast<int64_t>(warp - 2) * kChunks + c) * 8) * 32 + lane;
@@ -894,9 +901,12 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             tmem_ld_32x32b_x32(t_row + c * 32, acc);
             tmem_wait_ld();
             int4* dst = part_ptr(split, c);
+            const int64_t off = dst - reinterpret_cast<int4*>(p.partials);
+            if (SQ_GUARD(off >= 0 && off + 7 * 32 < p.partial_int4)) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              __stcg(dst + j * 32, make_int4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]));
+              for (int j = 0; j < 8; ++j)
+                __stcg(dst + j * 32, make_int4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]));
+            }
           }
         }
         tc_fence_before();
@@ -925,6 +935,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             for (int j = 0; j < 32; ++j) acc[j] = 0;
             for (int sidx = 0; sidx < p.splits; ++sidx) {
               const int4* src = part_ptr(sidx, c);
+              const int64_t off = src - reinterpret_cast<const int4*>(p.partials);
+              if (!SQ_GUARD(off >= 0 && off + 7 * 32 < p.partial_int4)) continue;
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
                 const int4 v = __ldcg(src + j * 32);
@@ -1027,7 +1039,7 @@ constexpr int kPlanSms = 148;  // planning is device-independent so workspace si
 constexpr int64_t kSwapMaxM = 64;  // token counts that fit one 64-column tile
 
 // Operand roles: up to 64 tokens (and no outlier product) swap the operands, so the weight
-// rows fill the 128-row MMA operand and the tokens one 64-column tile. Otherwise the tile
+// rows fill the 128-row MMA operand and the tokens one 32- or 64-column tile. Otherwise the tile
 // width is the widest of 256/128/64 whose tile count covers the SMs; 256-wide tiles become
 // 256 x 256 CTA-pair tiles when those still cover the SM pairs without padding rows (each
 // CTA then stages two thirds of the bytes per k-block of a one-CTA 128 x 256 tile).
@@ -1046,7 +1058,9 @@ Plan plan_gemm(int64_t M, int64_t N, int64_t K, bool outliers) {
   constexpr int wide = 256;
   Plan pl{swap, false, 64, 0, 0, 1, static_cast<int>(kb)};
   if (swap) {
-    pl.bn = 64;
+    // up to 32 tokens stage a 32-row activation tile (4 KB per k-block instead of 8 KB of
+    // mostly zero rows)
+    pl.bn = cols <= 32 ? 32 : 64;
   } else if (tiles(wide) >= kPlanSms) {
     pl.bn = wide;
     // CTA pairs when the 256-row tiles still give every pair of SMs a tile and add no
@@ -1147,10 +1161,12 @@ cudaError_t run(const GemmArgs& a, const Plan& pl, cudaStream_t stream, const ch
   p.num_units = pl.num_full + pl.tail_tiles * pl.splits;
   p.partials = nullptr;
   p.counters = nullptr;
+  p.partial_int4 = 0;
   if (pl.tail_tiles > 0) {
     p.partials = static_cast<int32_t*>(a.ws);
     p.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(a.ws) +
-                                            up256(sizeof(int32_t) * pl.tail_tiles * pl.splits * kBM * BN));
+                                            up256(static_cast<size_t>(pl.tail_tiles) * pl.splits * split_slot_bytes(BN)));
+    p.partial_int4 = static_cast<int64_t>(pl.tail_tiles) * pl.splits * split_slot_bytes(BN) / 16;
   }
   p.o_count = a.o_count;
   p.status = device_status_word();
@@ -1174,7 +1190,7 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, bool outliers) {
   if (gemv_applies(M, K, outliers)) return 0;
   const Plan pl = plan_gemm(M, N, K, outliers);
   if (pl.tail_tiles == 0) return 0;
-  return up256(sizeof(int32_t) * pl.tail_tiles * pl.splits * kBM * pl.bn) +
+  return up256(static_cast<size_t>(pl.tail_tiles) * pl.splits * split_slot_bytes(pl.bn)) +
          up256(sizeof(int32_t) * pl.tail_tiles * kEpiWarps);
 }
 
@@ -1207,12 +1223,15 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream, const char** why
     return run<256, false, 2, false, false, true>(a, pl, stream, why);
   }
   if (a.x_zero != nullptr) {
-    if (pl.swap) return run<64, false, 2, true, true>(a, pl, stream, why);
+    if (pl.swap)
+      return pl.bn == 32 ? run<32, false, 2, true, true>(a, pl, stream, why)
+                         : run<64, false, 2, true, true>(a, pl, stream, why);
     if (pl.bn == 256) return run<256, false, 2, false, true>(a, pl, stream, why);
     if (pl.bn == 128) return run<128, false, 2, false, true>(a, pl, stream, why);
     return run<64, false, 2, false, true>(a, pl, stream, why);
   }
-  if (pl.swap) return run<64, false, 2, true>(a, pl, stream, why);
+  if (pl.swap)
+    return pl.bn == 32 ? run<32, false, 2, true>(a, pl, stream, why) : run<64, false, 2, true>(a, pl, stream, why);
   if (pl.bn == 256) return run<256, false, 2, false>(a, pl, stream, why);
   if (pl.bn == 128) return run<128, false, 2, false>(a, pl, stream, why);
   return run<64, false, 2, false>(a, pl, stream, why);

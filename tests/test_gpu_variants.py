@@ -407,3 +407,24 @@ def test_strided_inputs_every_row_kernel():
     sq.sq_act_mean_std_threshold(X, 3.0, thr, None, sq.workspace(sq.SQ_OP_MEAN_STD_THRESHOLD, M, 0, K))
     sq.sq_sync_status()
     assert _ulps(host(thr), oracle.mean_std_threshold(Xc, 3.0)[0]).max() <= 1
+
+
+@pytest.mark.parametrize("norm", [sq.SQ_NORM_LAYER, sq.SQ_NORM_RMS])
+def test_norm_long_rows_strided(norm):
+    """The pipelined row groups copy whole rows through the leading dimension: a column slice
+    (K = 5008, ragged last chunks) of a matrix 8192 wide, starting 1024 columns in."""
+    rng = np.random.default_rng(57 + norm)
+    M, LD, K, off = 300, 8192, 5008, 1024
+    full = wl.f32_to_bf16_bits(rng.normal(0.4, 1.7, (M, LD)).astype(np.float32))
+    X = dev_bf16(full)[:, off:off + K]
+    Xc = np.ascontiguousarray(full[:, off:off + K])
+    g = wl.f32_to_bf16_bits(rng.uniform(0.5, 1.5, K).astype(np.float32))
+    b = wl.f32_to_bf16_bits(rng.normal(0, 0.2, K).astype(np.float32))
+    inv_s = rng.uniform(0.3, 2.0, K).astype(np.float32)
+    Xq, d, st = empty((M, K), torch.int8), empty(M, torch.float32), empty((M, 2), torch.float32)
+    sq.sq_norm_smooth_quant(X, norm, dev_bf16(g), dev_bf16(b), 1e-5, torch.from_numpy(inv_s).cuda(), Xq, d, st)
+    sq.sq_sync_status()
+    _, _, _, ost = oracle.norm_smooth_quant(Xc, norm, g, b, 1e-5, inv_s, with_stats=True)
+    assert _ulps(host(st), ost).max() <= 1
+    cq, cd, _ = oracle.norm_smooth_quant(Xc, norm, g, b, 1e-5, inv_s, stats=host(st))
+    assert np.array_equal(host(d), cd) and np.array_equal(host(Xq), cq)

@@ -111,6 +111,13 @@ def test_plan_invariants_and_workspace_agree():
         ws = sq.sq_workspace_size(sq.SQ_OP_INT8_GEMM_DEQUANT, M, N, K) if not outliers else None
         if ws is not None:
             assert (ws > 0) == (p["split_tiles"] > 0)
+            if p["split_tiles"]:
+                # each K-split unit stores, for each of the 8 epilogue warps, a 32 x 32 int32
+                # block per 32-column chunk of the warp's column half (the larger half when
+                # the tile has an odd number of chunks); one arrival counter per tile and warp
+                chunks = (p["bn"] // 32 + 1) // 2
+                slot = 8 * chunks * 32 * 32 * 4
+                assert ws >= p["split_tiles"] * p["splits"] * slot + p["split_tiles"] * 8 * 4, (M, N, K, p, ws)
 
 
 def test_bad_sizes_are_rejected():
